@@ -1,0 +1,180 @@
+"""Seeded synthetic workloads for the DSA hot path.
+
+This module only draws random inputs; it holds none of the method's
+arithmetic.  Both the CUDA path and the CPU oracle consume exactly the tensors
+it returns (the oracle gets host copies).  The one transformation it applies
+is input preparation for the FP8 workload: each token's values are divided by
+a per-token scale (amax / 448) and rounded to FP8-e4m3 by torch's cast; the
+codes and the fp32 scales then *are* the inputs of both sides.
+
+Shapes and value distributions follow the five workloads the DSA path is
+measured on (tiny integer prefill, integer prefill n=8192, FP8 prefill
+2x32768, decode batch 64 with ragged contexts 4096..65536, long prefill
+n=131072 in 8192-query chunks).  No dataset is involved.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import torch
+
+FP8_MAX = 448.0
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    kind: str                 # "prefill" or "decode"
+    B: int
+    n: int                    # tokens per sequence (prefill)
+    HI: int                   # indexer heads
+    dI: int                   # indexer head dim
+    k: int                    # top-k budget
+    H: int                    # attention query heads
+    Dqk: int                  # latent row width (key)
+    Dv: int                   # value width (first Dv columns of the latent row)
+    qk_dist: str              # "int" (uniform integers) or "normal"
+    qk_int_max: int = 0       # integers in [-qk_int_max, qk_int_max]
+    w_den: int = 0            # w = randint(-w_den, w_den) / w_den (int configs)
+    w_std: float = 0.1        # w ~ N(0, w_std^2) (float configs)
+    fp8: bool = False
+    chunk: int = 0            # prefill query chunk (0 = whole sequence)
+    seed: int = 0
+    L_min: int = 0            # decode context lengths uniform in [L_min, L_max]
+    L_max: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.Dqk)
+
+    @property
+    def integer_valued(self) -> bool:
+        return self.qk_dist == "int"
+
+
+TINY = Workload("tiny", "prefill", B=1, n=512, HI=4, dI=32, k=16, H=4, Dqk=64, Dv=64,
+                qk_dist="int", qk_int_max=4, w_den=4, seed=0)
+PREFILL = Workload("prefill", "prefill", B=1, n=8192, HI=64, dI=128, k=2048, H=16, Dqk=576,
+                   Dv=512, qk_dist="int", qk_int_max=3, w_den=16, seed=1)
+PREFILL_FP8 = Workload("prefill_fp8", "prefill", B=2, n=32768, HI=64, dI=128, k=2048, H=16,
+                       Dqk=576, Dv=512, qk_dist="normal", w_std=0.1, fp8=True, seed=2)
+DECODE = Workload("decode", "decode", B=64, n=0, HI=64, dI=128, k=2048, H=128, Dqk=576, Dv=512,
+                  qk_dist="normal", w_std=0.1, seed=3, L_min=4096, L_max=65536)
+LONG = Workload("long_prefill", "prefill", B=1, n=131072, HI=64, dI=128, k=2048, H=16, Dqk=576,
+                Dv=512, qk_dist="normal", w_std=0.1, chunk=8192, seed=4)
+
+ALL = {w.name: w for w in (TINY, PREFILL, PREFILL_FP8, DECODE, LONG)}
+
+
+def scaled(w: Workload, **changes) -> Workload:
+    """A copy of a workload with some sizes changed (for small parity cases)."""
+    return dataclasses.replace(w, **changes)
+
+
+def _gen(device, seed: int) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _ints(shape, lim, g, device):
+    return torch.randint(-lim, lim + 1, shape, generator=g, device=device)
+
+
+def quantize_fp8_per_token(x: torch.Tensor, group_dims: int):
+    """Per-token FP8-e4m3 input preparation: scale = amax / 448 over the last
+    ``group_dims`` dimensions, codes = round-to-nearest-even(x / scale)."""
+    red = tuple(range(x.dim() - group_dims, x.dim()))
+    amax = x.float().abs().amax(dim=red)
+    scale = torch.where(amax > 0, amax / FP8_MAX, torch.ones_like(amax))
+    y = x.float() / scale.reshape(scale.shape + (1,) * group_dims)
+    codes = y.clamp(-FP8_MAX, FP8_MAX).to(torch.float8_e4m3fn)
+    return codes, scale.float().contiguous()
+
+
+def make_prefill_inputs(w: Workload, device="cpu", n: Optional[int] = None,
+                        with_attention: bool = True) -> dict:
+    """All inputs of one prefill workload (whole sequence; chunks are views).
+
+    Returns a dict of tensors on ``device``:
+      qI [B,n,HI,dI] bf16 (or e4m3 codes + q_scale [B,n]),
+      kI [B,n,dI]    bf16 (or e4m3 codes + k_scale [B,n]),
+      w  [B,n,HI]    fp32,
+      q  [B,n,H,Dqk] bf16, latent [B,n,Dqk] bf16  (if with_attention).
+    """
+    n = w.n if n is None else n
+    g = _gen(device, w.seed)
+    out = {}
+    if w.qk_dist == "int":
+        out["qI"] = _ints((w.B, n, w.HI, w.dI), w.qk_int_max, g, device).to(torch.bfloat16)
+        out["kI"] = _ints((w.B, n, w.dI), w.qk_int_max, g, device).to(torch.bfloat16)
+        out["w"] = (_ints((w.B, n, w.HI), w.w_den, g, device).float() / w.w_den).contiguous()
+    else:
+        qI = torch.randn((w.B, n, w.HI, w.dI), generator=g, device=device)
+        kI = torch.randn((w.B, n, w.dI), generator=g, device=device)
+        if w.fp8:
+            out["qI"], out["q_scale"] = quantize_fp8_per_token(qI, 2)
+            out["kI"], out["k_scale"] = quantize_fp8_per_token(kI, 1)
+        else:
+            out["qI"] = qI.to(torch.bfloat16)
+            out["kI"] = kI.to(torch.bfloat16)
+        del qI, kI
+        out["w"] = (torch.randn((w.B, n, w.HI), generator=g, device=device) * w.w_std).float()
+    if with_attention:
+        out["q"] = torch.randn((w.B, n, w.H, w.Dqk), generator=g, device=device).to(torch.bfloat16)
+        out["latent"] = torch.randn((w.B, n, w.Dqk), generator=g, device=device).to(torch.bfloat16)
+    return out
+
+
+def decode_lengths(w: Workload, B: Optional[int] = None) -> torch.Tensor:
+    """Seeded context lengths L_b uniform in [L_min, L_max] (CPU generator)."""
+    B = w.B if B is None else B
+    g = _gen("cpu", w.seed)
+    return torch.randint(w.L_min, w.L_max + 1, (B,), generator=g)
+
+
+def make_decode_inputs(w: Workload, device="cpu", lengths: Optional[torch.Tensor] = None) -> dict:
+    """Inputs of one decode step: ragged caches plus the new token's queries.
+
+    Returns cu_seqlens int64 [B+1] (device), lengths (CPU),
+      qI [B,HI,dI] bf16, w [B,HI] fp32, kI_cache [sum L, dI] bf16,
+      q [B,H,Dqk] bf16, latent_cache [sum L, Dqk] bf16.
+    """
+    lengths = decode_lengths(w) if lengths is None else lengths
+    B = lengths.numel()
+    cu = torch.zeros(B + 1, dtype=torch.int64)
+    cu[1:] = torch.cumsum(lengths, 0)
+    total = int(cu[-1])
+    g = _gen(device, w.seed + 1000)
+    out = {"lengths": lengths, "cu_seqlens": cu.to(device)}
+    out["qI"] = torch.randn((B, w.HI, w.dI), generator=g, device=device).to(torch.bfloat16)
+    out["w"] = (torch.randn((B, w.HI), generator=g, device=device) * w.w_std).float()
+    out["kI_cache"] = torch.randn((total, w.dI), generator=g, device=device).to(torch.bfloat16)
+    out["q"] = torch.randn((B, w.H, w.Dqk), generator=g, device=device).to(torch.bfloat16)
+    out["latent_cache"] = torch.randn((total, w.Dqk), generator=g, device=device).to(torch.bfloat16)
+    return out
+
+
+def sample_rows(w: Workload, nrows: int = 256, n: Optional[int] = None, salt: int = 0):
+    """Seeded sample of query rows (b, i) for parity checks on large workloads.
+
+    Always includes rows 0, 1, k-2, k-1, k and the last row of batch 0 (and,
+    for chunked workloads, the first and last row of every chunk); the rest
+    are drawn uniformly.
+    """
+    n = w.n if n is None else n
+    g = torch.Generator().manual_seed(1234 + w.seed + salt)
+    must = {0, 1, w.k - 2, w.k - 1, w.k, n - 1}
+    if w.chunk:
+        for c0 in range(0, n, w.chunk):
+            must.add(c0)
+            must.add(min(n, c0 + w.chunk) - 1)
+    rows = {(0, i) for i in must if 0 <= i < n}
+    while len(rows) < min(nrows, w.B * n):
+        b = int(torch.randint(0, w.B, (1,), generator=g))
+        i = int(torch.randint(0, n, (1,), generator=g))
+        rows.add((b, i))
+    return sorted(rows)

@@ -1,0 +1,304 @@
+"""Plain CPU oracle for the DeepSeek Sparse Attention (DSA) hot path.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and
+the ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+module.  The CUDA library never calls it, and it shares no code, constant or
+helper with the CUDA library.
+
+Source: the page "2.2.1 · DSA 与索引器: 先召回 token, 再计算 Sparse MLA"
+(called "the DSA page" below), §1.1 eqs. (1)-(6), §2 (decode, quantised
+indexer key cache) and §3.1 eq. (18), §3.2 eqs. (19)-(20).
+
+Everything is float64 numpy.  Inputs are converted exactly to float64 first:
+bf16 values are exact in float64, and FP8-e4m3 codes are decoded by
+``e4m3_to_float64`` and multiplied by their fp32 scale (both exact in float64),
+so the quantisation is part of the input, not of the arithmetic.
+
+Readings of points the page leaves open (each is repeated where it is used):
+  * positions are 0-based and the current token is a candidate (eq. (2));
+  * ties in the score are broken toward the lower position;
+  * -0.0 is the same score as +0.0;
+  * unused slots of the fixed-width index tensor hold -1, after the valid ones;
+  * the attention of eq. (3) uses an explicit softmax scale; the key is the
+    whole latent row and the value is its first ``Dv`` columns; the rotary
+    part of query and latent arrives already rotated;
+  * a decode step's query is the last token of its sequence (position L-1)
+    and it scans all L cached keys, itself included.
+
+Parity status: every function here is pinned by ``tests/test_oracle.py``
+(worked example of §1.1, the min(k, t+1) rule, brute force on tiny inputs,
+library special cases, and the invariants of §3.1/§3.2).
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "e4m3_to_float64",
+    "dequantize",
+    "indexer_scores_row",
+    "indexer_scores",
+    "causal_topk_row",
+    "indexer_topk",
+    "selection_stats_row",
+    "sparse_attention_row",
+    "sparse_attention",
+    "decode_indexer_topk",
+    "decode_sparse_attention",
+]
+
+
+# ---------------------------------------------------------------------------
+# Inputs: exact conversion to float64
+# ---------------------------------------------------------------------------
+
+def e4m3_to_float64(codes) -> np.ndarray:
+    """Decode FP8 E4M3 ("fn" variant) byte codes to float64, exactly.
+
+    The DSA page (§2, quantised indexer key cache) says the indexer may run in
+    FP8 with a quantised key cache plus scales.  The format: 1 sign bit, 4
+    exponent bits with bias 7, 3 mantissa bits; exponent field 0 is subnormal
+    (value = m/8 * 2^-6); there is no infinity and only S.1111.111 is NaN.
+    """
+    c = np.asarray(codes).astype(np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    normal = sign * (1.0 + m / 8.0) * np.power(2.0, (e - 7).astype(np.float64))
+    subnormal = sign * (m / 8.0) * 2.0 ** -6
+    out = np.where(e == 0, subnormal, normal)
+    out = np.where((e == 0xF) & ((c & 0x7) == 0x7), np.nan, out)
+    return out
+
+
+def dequantize(codes, scale, axis_shape) -> np.ndarray:
+    """Dequantised value = e4m3 value x its per-token fp32 scale (float64).
+
+    ``scale`` has the leading shape of ``codes`` minus ``axis_shape`` trailing
+    dimensions (one scale per token, shared by the quantised group).
+    """
+    v = e4m3_to_float64(codes)
+    s = np.asarray(scale, dtype=np.float64)
+    return v * s.reshape(s.shape + (1,) * axis_shape)
+
+
+def _f64(x) -> np.ndarray:
+    """Exact conversion of a float array (numpy or torch, any float dtype)."""
+    if hasattr(x, "detach"):  # a torch tensor: go through float64 on the CPU
+        x = x.detach().to("cpu").double().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Eq. (1): Lightning Indexer score
+# ---------------------------------------------------------------------------
+
+def indexer_scores_row(q_t, k_hist, w_t) -> np.ndarray:
+    """Scores of one query against a list of keys, eq. (1) of the DSA page:
+
+        I[t, s] = sum_j  w[t, j] * ReLU( q[t, j] . k[s] )
+
+    q_t: [H_I, d_I] indexer queries of token t; k_hist: [m, d_I] keys;
+    w_t: [H_I] real-valued (possibly negative) head weights.
+    Returns [m] float64 with -0.0 replaced by +0.0.
+    """
+    q_t = _f64(q_t)
+    k_hist = _f64(k_hist)
+    w_t = _f64(w_t)
+    dots = k_hist @ q_t.T                     # [m, H_I]: q[t,j] . k[s]
+    relu = np.maximum(dots, 0.0)              # per-head ReLU
+    scores = relu @ w_t                       # weighted sum over heads
+    return scores + 0.0                       # -0.0 -> +0.0
+
+
+def indexer_scores(q, k, w, q_offset: int = 0) -> np.ndarray:
+    """Dense causal score matrix for a prefill chunk (DSA page §1.1 shapes).
+
+    q: [B, nq, H_I, d_I], k: [B, kv_len, d_I], w: [B, nq, H_I].
+    Query row i of the chunk sits at absolute position t = q_offset + i and
+    sees keys 0 <= s <= t.  Returns [B, nq, kv_len] float64, -inf where s > t.
+    """
+    q = _f64(q)
+    k = _f64(k)
+    w = _f64(w)
+    B, nq = q.shape[0], q.shape[1]
+    kv_len = k.shape[1]
+    out = np.full((B, nq, kv_len), -np.inf)
+    for b in range(B):
+        for i in range(nq):
+            t = q_offset + i
+            out[b, i, : t + 1] = indexer_scores_row(q[b, i], k[b, : t + 1], w[b, i])
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Eq. (2): causal top-k with a fixed-width, -1 padded index tensor
+# ---------------------------------------------------------------------------
+
+def causal_topk_row(scores_row, t: int, k: int) -> np.ndarray:
+    """S_t = TopK({I[t, s] : 0 <= s <= t}, min(k, t + 1)), eq. (2).
+
+    Positions are 0-based and include the current token.  Ties go to the
+    lower position.  The result has width k: the min(k, t+1) selected
+    positions in rank order (score descending, then position ascending),
+    followed by -1 in every unused slot.
+    """
+    s = np.asarray(scores_row, dtype=np.float64)[: t + 1] + 0.0
+    m = min(k, t + 1)
+    # A stable sort of -score keeps equal scores in ascending position order.
+    order = np.argsort(-s, kind="stable")[:m]
+    out = np.full(k, -1, dtype=np.int64)
+    out[:m] = order
+    return out
+
+
+def selection_stats_row(scores_row, t: int, k: int) -> dict:
+    """Cut-off quantities of one row for tolerance-aware comparison.
+
+    tau       -- the score at rank m = min(k, t+1) (the last one kept);
+    n_above   -- how many scores are strictly above tau (all must be kept);
+    margin    -- Delta_k = s_(k) - s_(k+1), eq. (18) of the DSA page §3.1
+                 (+inf when nothing is left out);
+    max_abs   -- the largest |score| in the row.
+    """
+    s = np.asarray(scores_row, dtype=np.float64)[: t + 1] + 0.0
+    m = min(k, t + 1)
+    srt = np.sort(s)[::-1]
+    tau = srt[m - 1]
+    nxt = srt[m] if m < s.size else -np.inf
+    return {
+        "tau": float(tau),
+        "n_above": int(np.count_nonzero(s > tau)),
+        "margin": float(tau - nxt),
+        "max_abs": float(np.max(np.abs(s))),
+    }
+
+
+def indexer_topk(q, k, w, topk: int, q_offset: int = 0, rows=None) -> np.ndarray:
+    """Eq. (1) then eq. (2) for a prefill chunk.  Returns [B, nq, topk] int64.
+
+    ``rows`` optionally restricts the work to a list of (b, i) query rows;
+    the other rows of the result are left at -2 (not computed).
+    """
+    q = _f64(q)
+    k = _f64(k)
+    w = _f64(w)
+    B, nq = q.shape[0], q.shape[1]
+    out = np.full((B, nq, topk), -2, dtype=np.int64)
+    todo = rows if rows is not None else [(b, i) for b in range(B) for i in range(nq)]
+    for b, i in todo:
+        t = q_offset + i
+        sc = indexer_scores_row(q[b, i], k[b, : t + 1], w[b, i])
+        out[b, i] = causal_topk_row(sc, t, topk)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Eq. (3): sparse attention over the selected latent rows
+# ---------------------------------------------------------------------------
+
+def sparse_attention_row(q_t, latent, sel, scale: float, dv: int):
+    """u_t = Attn(h_t, {c_s : s in S_t}), eq. (3) of the DSA page, one token.
+
+    The selector only chooses rows; the attention computes its own logits
+    (the indexer scores are not reused, §1.1).  Every query head attends the
+    same selected set (the key is shared by all heads, §1.1).
+
+    q_t: [H, Dqk] query heads; latent: [kv_len, Dqk] latent cache rows c_s;
+    sel: selected positions, -1 entries are ignored.
+    logits z[h, s] = scale * q_t[h] . c_s;  p = softmax over the selected s;
+    out[h] = sum_s p[h, s] * c_s[:dv];  lse[h] = log sum_s exp z[h, s].
+    With no valid entry the output is 0 and lse is -inf.
+    """
+    q_t = _f64(q_t)
+    latent = _f64(latent)
+    sel = np.asarray(sel, dtype=np.int64)
+    sel = sel[sel >= 0]
+    H = q_t.shape[0]
+    if sel.size == 0:
+        return np.zeros((H, dv)), np.full(H, -np.inf)
+    c = latent[sel]                                  # [m, Dqk]
+    z = scale * (q_t @ c.T)                          # [H, m]
+    zmax = z.max(axis=1, keepdims=True)
+    e = np.exp(z - zmax)
+    denom = e.sum(axis=1, keepdims=True)
+    p = e / denom
+    out = p @ c[:, :dv]                              # [H, dv]
+    lse = (zmax + np.log(denom))[:, 0]
+    return out, lse
+
+
+def sparse_attention(q, latent, idx, scale: float, dv: int, rows=None):
+    """Eq. (3) for a prefill chunk.
+
+    q: [B, nq, H, Dqk], latent: [B, kv_len, Dqk], idx: [B, nq, k] (-1 padded).
+    Returns out [B, nq, H, dv] and lse [B, nq, H] (float64).  ``rows``
+    optionally restricts the work to a list of (b, i) rows (others are NaN).
+    """
+    q = _f64(q)
+    latent = _f64(latent)
+    idx = np.asarray(idx.cpu() if hasattr(idx, "cpu") else idx, dtype=np.int64)
+    B, nq, H = q.shape[0], q.shape[1], q.shape[2]
+    out = np.full((B, nq, H, dv), np.nan)
+    lse = np.full((B, nq, H), np.nan)
+    todo = rows if rows is not None else [(b, i) for b in range(B) for i in range(nq)]
+    for b, i in todo:
+        out[b, i], lse[b, i] = sparse_attention_row(q[b, i], latent[b], idx[b, i], scale, dv)
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# Decode step (DSA page §2: one new query scans every cached indexer key)
+# ---------------------------------------------------------------------------
+
+def decode_indexer_topk(q, w, k_cache, cu_seqlens, topk: int, with_scores: bool = False):
+    """One decode step of the indexer and selector for a batch of sequences.
+
+    q: [B, H_I, d_I] the new token's indexer queries; w: [B, H_I];
+    k_cache: [sum L, d_I] ragged indexer key cache, sequence b in rows
+    cu_seqlens[b] .. cu_seqlens[b+1]-1; L_b includes the new token, whose
+    position is t = L_b - 1.  Returns idx [B, topk] of positions local to
+    each sequence (and the per-sequence score rows if asked).
+    """
+    q = _f64(q)
+    w = _f64(w)
+    k_cache = _f64(k_cache)
+    cu = np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int64)
+    B = q.shape[0]
+    out = np.full((B, topk), -1, dtype=np.int64)
+    rows = []
+    for b in range(B):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        sc = indexer_scores_row(q[b], k_cache[lo:hi], w[b])
+        out[b] = causal_topk_row(sc, hi - lo - 1, topk)
+        rows.append(sc)
+    return (out, rows) if with_scores else out
+
+
+def decode_sparse_attention(q, latent_cache, cu_seqlens, idx, scale: float, dv: int):
+    """Eq. (3) for a decode step: every query head of a sequence attends the
+    same selected rows of that sequence's latent cache (the MQA form of §2).
+
+    q: [B, H, Dqk]; latent_cache: [sum L, Dqk]; idx: [B, k] local positions.
+    Returns out [B, H, dv], lse [B, H].
+    """
+    q = _f64(q)
+    latent_cache = _f64(latent_cache)
+    cu = np.asarray(cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int64)
+    idx = np.asarray(idx.cpu() if hasattr(idx, "cpu") else idx, dtype=np.int64)
+    B, H = q.shape[0], q.shape[1]
+    out = np.zeros((B, H, dv))
+    lse = np.zeros((B, H))
+    for b in range(B):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        out[b], lse[b] = sparse_attention_row(q[b], latent_cache[lo:hi], idx[b], scale, dv)
+    return out, lse
+
+
+def softmax_scale_default(dqk: int) -> float:
+    """Default attention scale 1/sqrt(Dqk) (the dense-attention scale written
+    on the page "2 · 动态路由", §3.1); the page on DSA leaves it implicit."""
+    return 1.0 / math.sqrt(dqk)

@@ -1,0 +1,349 @@
+"""Pins of the CPU oracle against facts fixed by the DSA page and by mathematics.
+
+None of these tests re-run the oracle's own formula: each compares it with a
+printed value (the page's worked example), an exact brute force written with
+different arithmetic (Python integers / fractions), a library routine for a
+special case (torch's scaled_dot_product_attention, torch's FP8 cast), or an
+invariant the page states (order invariance §3.1, renormalisation eq. (19)
+and bound eq. (20) §3.2).
+"""
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _worked():
+    with open(os.path.join(GOLDEN, "worked_example.json")) as f:
+        return json.load(f)
+
+
+# --------------------------------------------------------------------------
+# FP8 decoding
+# --------------------------------------------------------------------------
+
+def test_e4m3_decode_known_codes():
+    v = O.e4m3_to_float64(np.array([0x38, 0x7E, 0x01, 0x08, 0xB8, 0x00, 0x80, 0x7F], dtype=np.uint8))
+    assert v[0] == 1.0
+    assert v[1] == 448.0            # largest finite e4m3
+    assert v[2] == 2.0 ** -9        # smallest subnormal
+    assert v[3] == 2.0 ** -6        # smallest normal
+    assert v[4] == -1.0
+    assert v[5] == 0.0 and v[6] == 0.0
+    assert math.isnan(v[7])
+
+
+def test_e4m3_decode_matches_torch_cast():
+    codes = torch.arange(256, dtype=torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = O.e4m3_to_float64(codes.numpy())
+    finite = ~np.isnan(ref)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert np.array_equal(got[finite], ref[finite])
+
+
+# --------------------------------------------------------------------------
+# Worked example of §1.1 (eqs. (4)-(6) and the text after them)
+# --------------------------------------------------------------------------
+
+def test_worked_example_scores():
+    g = _worked()
+    s = O.indexer_scores_row(np.array(g["q"], float), np.array(g["keys"], float), np.array(g["w"]))
+    assert s.tolist() == g["scores"]
+    # the per-head ReLU table printed on the page
+    dots = np.array(g["keys"], float) @ np.array(g["q"], float).T
+    assert np.maximum(dots, 0).tolist() == g["per_head_relu"]
+
+
+def test_worked_example_selection():
+    g = _worked()
+    s = np.array(g["scores"])
+    t = len(s) - 1                       # the query is the third token (0-based t = 2)
+    idx = O.causal_topk_row(s, t, g["k"])
+    assert sorted(idx.tolist()) == g["selected_positions_0based"]
+    assert [p + 1 for p in sorted(idx.tolist())] == g["selected_positions_1based"]
+    # derived from the tie rule (lower position wins) and eq. (2)
+    assert O.causal_topk_row(s, t, 1).tolist() == [0]
+    assert O.causal_topk_row(s, t, 3).tolist() == [0, 1, 2]
+    assert O.causal_topk_row(s, t, 5).tolist() == [0, 1, 2, -1, -1]
+
+
+def _example_attention_inputs(g):
+    # Embedding of the printed logits: c_s = (v_s | a_s), q = (0, 0 | 1), scale 1,
+    # so scale * q . c_s = a_s exactly and the value is the first 2 columns.
+    a = g["attention_logits"] + [g["miss_case_logit_position3"]]
+    v = g["attention_values"] + [[7.0, -5.0]]      # any value for position 3
+    latent = np.array([vi + [ai] for vi, ai in zip(v, a)], float)
+    q = np.array([[0.0, 0.0, 1.0]])
+    return q, latent
+
+
+def test_worked_example_attention():
+    g = _worked()
+    q, latent = _example_attention_inputs(g)
+    out, lse = O.sparse_attention_row(q, latent, np.array(g["selected_positions_0based"]), 1.0, 2)
+    tol = 0.5 * 10 ** -g["printed_decimals"]
+    e = np.exp(np.array(g["attention_logits"]))
+    weights = e / e.sum()
+    assert np.allclose(weights, g["attention_weights_printed"], atol=tol, rtol=0)
+    assert np.allclose(out[0], g["attention_output_printed"], atol=tol, rtol=0)
+    assert abs(out[0, 0] - 0.537883) < 1e-6 and abs(out[0, 1] - 2.193176) < 1e-6
+    assert abs(lse[0] - math.log(math.exp(0.2) + math.exp(1.2))) < 1e-12
+
+
+def test_worked_example_miss_case_renormalises():
+    """If position 3 had the largest full logit, the sparse softmax still only
+    renormalises over {1, 2} (1-based): the output is unchanged by position 3."""
+    g = _worked()
+    q, latent = _example_attention_inputs(g)
+    sparse, _ = O.sparse_attention_row(q, latent, np.array([0, 1, -1]), 1.0, 2)
+    dense, _ = O.sparse_attention_row(q, latent, np.array([0, 1, 2]), 1.0, 2)
+    assert np.allclose(sparse[0], g["attention_output_printed"], atol=5e-4)
+    assert not np.allclose(dense, sparse, atol=1e-2)
+
+
+# --------------------------------------------------------------------------
+# Eq. (1) special cases and invariants
+# --------------------------------------------------------------------------
+
+def test_single_head_unit_weight_is_relu_of_dot():
+    rng = np.random.default_rng(0)
+    q = rng.standard_normal((1, 16))
+    k = rng.standard_normal((40, 16))
+    s_pos = O.indexer_scores_row(q, k, np.array([1.0]))
+    s_neg = O.indexer_scores_row(q, k, np.array([-1.0]))
+    for j in range(40):
+        d = float(np.dot(q[0], k[j]))
+        assert s_pos[j] == pytest.approx(max(d, 0.0), rel=1e-12, abs=1e-12)
+        assert s_neg[j] == pytest.approx(-max(d, 0.0), rel=1e-12, abs=1e-12)
+
+
+def test_scores_are_linear_in_head_weights():
+    rng = np.random.default_rng(1)
+    q = rng.standard_normal((8, 32))
+    k = rng.standard_normal((50, 32))
+    w1, w2 = rng.standard_normal(8), rng.standard_normal(8)
+    s1 = O.indexer_scores_row(q, k, w1)
+    s2 = O.indexer_scores_row(q, k, w2)
+    assert np.allclose(O.indexer_scores_row(q, k, w1 + w2), s1 + s2, atol=1e-12)
+    assert np.allclose(O.indexer_scores_row(q, k, -3.0 * w1), -3.0 * s1, atol=1e-12)
+
+
+def test_relu_drops_negative_dots_and_negative_weights_subtract():
+    # every key has a negative dot product with head 0 and positive with head 1
+    q = np.array([[1.0, 0.0], [0.0, 1.0]])
+    k = np.array([[-1.0, 2.0], [-3.0, 0.5]])
+    s = O.indexer_scores_row(q, k, np.array([5.0, -1.0]))
+    assert s.tolist() == [-2.0, -0.5]
+    s0 = O.indexer_scores_row(q, k, np.array([5.0, 0.0]))
+    assert s0.tolist() == [0.0, 0.0] and not np.signbit(s0).any()
+
+
+def test_positive_head_scaling_and_query_scaling_commute_with_relu():
+    # ReLU(c x) = c ReLU(x) for c > 0: scaling a head's query by c equals
+    # scaling its weight by c (this is what lets FP8 query scales fold into w).
+    rng = np.random.default_rng(2)
+    q = rng.standard_normal((4, 16))
+    k = rng.standard_normal((30, 16))
+    w = rng.standard_normal(4)
+    c = np.array([0.5, 2.0, 3.0, 0.25])
+    a = O.indexer_scores_row(q * c[:, None], k, w)
+    b = O.indexer_scores_row(q, k, w * c)
+    assert np.allclose(a, b, atol=1e-12)
+
+
+def test_prefill_scores_causal_mask_and_offset():
+    rng = np.random.default_rng(3)
+    B, n, HI, dI = 2, 12, 3, 8
+    q = rng.integers(-3, 4, (B, n, HI, dI)).astype(float)
+    k = rng.integers(-3, 4, (B, n, dI)).astype(float)
+    w = rng.integers(-4, 5, (B, n, HI)) / 4.0
+    full = O.indexer_scores(q, k, w)
+    for b in range(B):
+        for t in range(n):
+            assert np.all(np.isneginf(full[b, t, t + 1:]))
+            assert np.all(np.isfinite(full[b, t, : t + 1]))
+    # a chunk of queries starting at position 5 sees the same rows
+    part = O.indexer_scores(q[:, 5:9], k, w[:, 5:9], q_offset=5)
+    assert np.array_equal(part, full[:, 5:9])
+
+
+# --------------------------------------------------------------------------
+# Eq. (2): selection
+# --------------------------------------------------------------------------
+
+def _brute_scores_fraction(q, k, w_num, w_den):
+    """Exact eq. (1) with Python integers and Fractions, explicit loops."""
+    HI, dI = len(q), len(q[0])
+    out = []
+    for ks in k:
+        total = Fraction(0)
+        for j in range(HI):
+            d = 0
+            for x in range(dI):
+                d += int(q[j][x]) * int(ks[x])
+            if d > 0:
+                total += Fraction(int(w_num[j]), w_den) * d
+        out.append(total)
+    return out
+
+
+def _brute_select(scores, k):
+    """Repeatedly take the best remaining position: larger score first, and
+    among equal scores the lower position (explicit loops, no sorting)."""
+    remaining = list(range(len(scores)))
+    chosen = []
+    while remaining and len(chosen) < k:
+        best = remaining[0]
+        for p in remaining[1:]:
+            if scores[p] > scores[best]:
+                best = p
+        chosen.append(best)
+        remaining.remove(best)
+    return chosen + [-1] * (k - len(chosen))
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_selection_matches_brute_force_with_ties(seed):
+    rng = np.random.default_rng(100 + seed)
+    n, HI, dI, w_den = 24, 3, 4, 4
+    q = rng.integers(-2, 3, (n, HI, dI))
+    k = rng.integers(-2, 3, (n, dI))
+    w_num = rng.integers(-4, 5, (n, HI))
+    for topk in (1, 3, 8, 30):
+        got = O.indexer_topk(q[None].astype(float), k[None].astype(float),
+                             (w_num / w_den)[None], topk)[0]
+        for t in range(n):
+            exact = _brute_scores_fraction(q[t], k[: t + 1], w_num[t], w_den)
+            assert got[t].tolist() == _brute_select(exact, topk), (seed, topk, t)
+
+
+def test_short_history_rule():
+    rng = np.random.default_rng(5)
+    n, topk = 20, 8
+    q = rng.standard_normal((1, n, 2, 4))
+    k = rng.standard_normal((1, n, 4))
+    w = rng.standard_normal((1, n, 2))
+    idx = O.indexer_topk(q, k, w, topk)[0]
+    for t in range(n):
+        m = min(topk, t + 1)
+        assert sorted(idx[t, :m].tolist()) == sorted(set(idx[t, :m].tolist()))
+        assert all(0 <= p <= t for p in idx[t, :m])
+        assert np.all(idx[t, m:] == -1)
+        if t + 1 <= topk:
+            assert sorted(idx[t, :m].tolist()) == list(range(t + 1))
+
+
+def test_selection_invariant_under_shift_and_positive_scale():
+    rng = np.random.default_rng(6)
+    s = rng.integers(-5, 6, 60).astype(float)      # many ties
+    base = O.causal_topk_row(s, 59, 17)
+    assert np.array_equal(O.causal_topk_row(2.5 * s + 11.0, 59, 17), base)
+    # -0.0 and +0.0 are the same score
+    z = np.array([0.0, -0.0, 0.0, -0.0])
+    assert O.causal_topk_row(z, 3, 2).tolist() == [0, 1]
+
+
+def test_selection_stats_margin():
+    s = np.array([3.0, 1.0, 5.0, 1.0, 2.0])
+    st = O.selection_stats_row(s, 4, 3)
+    assert st["tau"] == 2.0 and st["n_above"] == 2 and st["margin"] == 1.0
+    st = O.selection_stats_row(s, 4, 4)
+    assert st["tau"] == 1.0 and st["n_above"] == 3 and st["margin"] == 0.0
+    st = O.selection_stats_row(s, 4, 5)
+    assert st["margin"] == math.inf
+
+
+# --------------------------------------------------------------------------
+# Eq. (3): attention
+# --------------------------------------------------------------------------
+
+def test_full_budget_equals_causal_dense_attention():
+    """With k >= t+1 every position is selected and eq. (3) is ordinary causal
+    attention with one shared key/value row per position (MQA form)."""
+    rng = np.random.default_rng(7)
+    n, H, Dqk, Dv = 10, 3, 16, 12
+    q = rng.standard_normal((1, n, H, Dqk))
+    lat = rng.standard_normal((1, n, Dqk))
+    scale = 0.3
+    idx = np.stack([np.concatenate([np.arange(t + 1)[::-1], -np.ones(n - t - 1, int)]) for t in range(n)])
+    out, lse = O.sparse_attention(q, lat, idx[None], scale, Dv)
+    qt = torch.from_numpy(q[0]).permute(1, 0, 2)               # [H, n, Dqk]
+    kt = torch.from_numpy(lat[0])[None].expand(H, n, Dqk)
+    vt = torch.from_numpy(lat[0, :, :Dv])[None].expand(H, n, Dv)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True, scale=scale)
+    assert np.allclose(out[0], ref.permute(1, 0, 2).numpy(), atol=1e-12)
+    logits = scale * torch.einsum("hqd,hkd->hqk", qt, kt)
+    mask = torch.ones(n, n, dtype=torch.bool).tril()
+    ref_lse = torch.logsumexp(logits.masked_fill(~mask, -math.inf), dim=-1)
+    assert np.allclose(lse[0], ref_lse.permute(1, 0).numpy(), atol=1e-12)
+
+
+def test_sparse_renormalisation_identity_and_bound():
+    """Eq. (19): the sparse output equals sum_{j in S} (a_j / M_k) v_j with a the
+    dense softmax; eq. (20): |o - o~| <= 2 (1 - M_k) V with V = max |v_j|."""
+    rng = np.random.default_rng(8)
+    m, Dqk, Dv = 40, 8, 6
+    lat = rng.standard_normal((m, Dqk)) * 1.5
+    q = rng.standard_normal((1, Dqk))
+    sel = rng.choice(m, 15, replace=False)
+    dense, _ = O.sparse_attention_row(q, lat, np.arange(m), 1.0, Dv)
+    sparse, _ = O.sparse_attention_row(q, lat, sel, 1.0, Dv)
+    z = lat @ q[0]
+    a = np.exp(z - z.max())
+    a /= a.sum()
+    M = a[sel].sum()
+    v = lat[:, :Dv]
+    renorm = (a[sel, None] / M * v[sel]).sum(axis=0)
+    assert np.allclose(sparse[0], renorm, atol=1e-12)
+    V = np.linalg.norm(v, axis=1).max()
+    assert np.linalg.norm(dense[0] - sparse[0]) <= 2 * (1 - M) * V + 1e-12
+
+
+def test_attention_ignores_padding_and_slot_order():
+    rng = np.random.default_rng(9)
+    lat = rng.standard_normal((30, 8))
+    q = rng.standard_normal((2, 8))
+    sel = np.array([4, 17, 2, 9])
+    a, la = O.sparse_attention_row(q, lat, sel, 0.5, 5)
+    b, lb = O.sparse_attention_row(q, lat, np.array([9, -1, 2, 17, -1, 4]), 0.5, 5)
+    assert np.allclose(a, b, atol=1e-13) and np.allclose(la, lb, atol=1e-13)
+    e, le = O.sparse_attention_row(q, lat, np.array([-1, -1]), 0.5, 5)
+    assert np.all(e == 0) and np.all(np.isneginf(le))
+
+
+# --------------------------------------------------------------------------
+# Decode = last row of prefill
+# --------------------------------------------------------------------------
+
+def test_decode_equals_last_prefill_row():
+    rng = np.random.default_rng(10)
+    lens = [7, 13, 5]
+    HI, dI, H, Dqk, Dv, topk = 2, 4, 3, 8, 6, 4
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    kc = rng.integers(-3, 4, (cu[-1], dI)).astype(float)
+    lat = rng.standard_normal((cu[-1], Dqk))
+    qI = rng.integers(-3, 4, (3, HI, dI)).astype(float)
+    w = rng.integers(-4, 5, (3, HI)) / 4.0
+    q = rng.standard_normal((3, H, Dqk))
+    idx = O.decode_indexer_topk(qI, w, kc, cu, topk)
+    out, lse = O.decode_sparse_attention(q, lat, cu, idx, 0.4, Dv)
+    for b, L in enumerate(lens):
+        lo = cu[b]
+        qpre = np.zeros((1, L, HI, dI))
+        qpre[0, -1] = qI[b]
+        wpre = np.zeros((1, L, HI))
+        wpre[0, -1] = w[b]
+        pre = O.indexer_topk(qpre, kc[None, lo:lo + L], wpre, topk, rows=[(0, L - 1)])
+        assert pre[0, L - 1].tolist() == idx[b].tolist()
+        o2, l2 = O.sparse_attention_row(q[b], lat[lo:lo + L], idx[b], 0.4, Dv)
+        assert np.allclose(out[b], o2) and np.allclose(lse[b], l2)
