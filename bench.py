@@ -1,0 +1,595 @@
+"""Benchmark of the DSA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl b200|reference]
+
+One step = the whole hot path over one batch of synthetic, HBM-resident input:
+the fused Lightning Indexer + causal top-k (eqs. (1)-(2) of the page
+"2.2.1 · DSA 与索引器") followed by sparse attention over the selected latent
+rows (eq. (3)).  The default workload is the integer-valued prefill
+(B=1, n=8192, HI=64, dI=128, k=2048, 16 heads, latent 576/512); the metric is
+query tokens per second.  --workload decode|prefill_fp8|long_prefill|tiny
+selects the other workloads.
+
+Timing: W warm-up steps, then exactly K steps, each bracketed by CUDA events
+on the launching stream; L2 is flushed (a 256 MiB write) before every timed
+step, outside the events.  Per-kernel events give the roofline of the
+dominant kernel.  Under torchrun every rank runs its own batch (weak
+scaling, no collective on the data path); rank 0 prints the max over ranks.
+
+--impl reference times the CPU oracle (float64 numpy) on a bounded sample of
+the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from learned_token_indexer_b200 import workloads as W  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = {
+    "prefill": ("prefill query-tokens/s (indexer+top-k+sparse attn)", "query-tokens/s"),
+    "decode": ("decode tokens/s (indexer scan+top-k+sparse attn)", "tokens/s"),
+}
+
+
+# ----------------------------------------------------------------------------
+# helpers
+# ----------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "learned_token_indexer_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+KERNEL_SOURCES = {
+    "indexer_topk_prefill": ["indexer_topk_prefill.cu", "indexer_common.cuh", "select.cuh", "sm100.cuh"],
+    "sparse_attn": ["sparse_attn.cu"],
+    "indexer_scan": ["indexer_scan.cu", "indexer_common.cuh", "sm100.cuh"],
+    "topk_rows": ["topk.cu", "select.cuh"],
+}
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    summary is missing or the kernel source changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel}:{workload}")
+    if not e or e.get("source_hash") != kernel_source_hash(KERNEL_SOURCES[kernel]):
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"dsa_clocks_{os.getpid()}_{gpu_index}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(parts)
+                except ValueError:
+                    pass
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def count_pairs_needed(n_rows_first: int, n_rows: int, k: int) -> int:
+    """(t, s) score pairs eq. (2) needs: rows with t + 1 > k score all t + 1
+    keys; rows with t + 1 <= k select every key without a score."""
+    tot = 0
+    lo = max(n_rows_first, k)
+    hi = n_rows_first + n_rows       # rows t in [n_rows_first, hi)
+    if hi > lo:
+        tot = (hi * (hi + 1) - lo * (lo + 1)) // 2
+    return tot
+
+
+def selected_entries(t0: int, n_rows: int, k: int) -> int:
+    return sum(min(k, t + 1) for t in range(t0, t0 + n_rows))
+
+
+# ----------------------------------------------------------------------------
+# the B200 arm
+# ----------------------------------------------------------------------------
+
+class PrefillRun:
+    def __init__(self, w: W.Workload, device):
+        import learned_token_indexer_b200 as dsa
+        self.dsa, self.w, self.dev = dsa, w, device
+        self.d = W.make_prefill_inputs(w, device)
+        self.ws_idx = dsa.Workspace(device)
+        self.ws_att = dsa.Workspace(device)
+        self.idx = torch.empty((w.B, w.n, w.k), dtype=torch.int32, device=device)
+        self.out = torch.empty((w.B, w.n, w.H, w.Dv), dtype=torch.bfloat16, device=device)
+        self.chunk = w.chunk or w.n
+        self.kw = {}
+        if w.fp8:
+            self.kw = dict(q_scale=self.d["q_scale"], k_scale=self.d["k_scale"])
+        self.launches_per_step = 0
+
+    def step(self, ev=None):
+        dsa, w, d = self.dsa, self.w, self.d
+        launches = 0
+        for c0 in range(0, w.n, self.chunk):
+            c1 = min(w.n, c0 + self.chunk)
+            sl = (slice(None), slice(c0, c1))
+            kw = dict(self.kw)
+            if w.fp8 and self.chunk != w.n:
+                kw["q_scale"] = self.kw["q_scale"][sl].contiguous()
+            if ev is not None:
+                ev["idx"][0].append(self._rec())
+            dsa.indexer_topk_prefill(d["qI"][sl], d["kI"], d["w"][sl], w.k, q_offset=c0, idx_out=self.idx[sl],
+                                     workspace=self.ws_idx, **kw)
+            if ev is not None:
+                ev["idx"][1].append(self._rec())
+            dsa.sparse_attn_prefill(d["q"][sl], d["latent"], self.idx[sl], w.Dv, scale=w.scale, out=self.out[sl],
+                                    workspace=self.ws_att)
+            if ev is not None:
+                ev["attn"][1].append(self._rec())
+            triv = c0 < w.k
+            launches += 2 + (1 if triv else 0)
+        self.launches_per_step = launches
+
+    @staticmethod
+    def _rec():
+        e = torch.cuda.Event(enable_timing=True)
+        e.record()
+        return e
+
+    def rows(self):
+        return self.w.B * self.w.n
+
+    def kernel_work(self):
+        w = self.w
+        pairs = 0
+        ent = 0
+        for c0 in range(0, w.n, self.chunk):
+            c1 = min(w.n, c0 + self.chunk)
+            pairs += count_pairs_needed(c0, c1 - c0, w.k)
+        ent = selected_entries(0, w.n, w.k)
+        return {
+            "indexer_topk_prefill": {"flops": 2 * w.HI * w.dI * w.B * pairs, "unit": "TFLOP/s",
+                                     "per_unit": f"2*HI*dI = {2 * w.HI * w.dI} FLOP per scored (t,s) pair",
+                                     "units": w.B * pairs},
+            "sparse_attn": {"flops": 2 * w.H * w.B * ent * (w.Dqk + w.Dv), "unit": "TFLOP/s",
+                            "per_unit": f"2*H*(Dqk+Dv) = {2 * w.H * (w.Dqk + w.Dv)} FLOP per selected entry",
+                            "units": w.B * ent},
+        }
+
+    def host_inputs(self):
+        return {k: v.cpu().pin_memory() for k, v in self.d.items() if isinstance(v, torch.Tensor)}
+
+    def load_inputs(self, host):
+        for k, v in host.items():
+            self.d[k].copy_(v, non_blocking=True)
+
+    def result(self):
+        return self.out
+
+
+class DecodeRun:
+    def __init__(self, w: W.Workload, device):
+        import learned_token_indexer_b200 as dsa
+        self.dsa, self.w, self.dev = dsa, w, device
+        self.d = W.make_decode_inputs(w, device)
+        self.lengths = self.d["lengths"]
+        self.total = int(self.lengths.sum())
+        self.maxlen = int(self.lengths.max())
+        self.ws_idx = dsa.Workspace(device)
+        self.ws_att = dsa.Workspace(device)
+        self.idx = torch.empty((w.B, w.k), dtype=torch.int32, device=device)
+        self.out = torch.empty((w.B, w.H, w.Dv), dtype=torch.bfloat16, device=device)
+        self.launches_per_step = 3
+
+    def step(self, ev=None):
+        dsa, w, d = self.dsa, self.w, self.d
+        if ev is not None:
+            ev["idx"][0].append(PrefillRun._rec())
+        dsa.indexer_topk_decode(d["qI"], d["w"], d["kI_cache"], d["cu_seqlens"], w.k, self.total, self.maxlen,
+                                idx_out=self.idx, workspace=self.ws_idx)
+        if ev is not None:
+            ev["idx"][1].append(PrefillRun._rec())
+        dsa.sparse_attn_decode(d["q"], d["latent_cache"], d["cu_seqlens"], self.idx, w.Dv, self.total,
+                               scale=w.scale, out=self.out, workspace=self.ws_att)
+        if ev is not None:
+            ev["attn"][1].append(PrefillRun._rec())
+
+    def rows(self):
+        return self.w.B
+
+    def kernel_work(self):
+        w = self.w
+        scan_bytes = self.total * w.dI * 2 + w.B * w.HI * (w.dI * 2 + 4) + self.total * 4 * 2
+        gather = w.B * w.k * w.Dqk * 2
+        return {
+            "indexer_topk_decode": {"bytes": scan_bytes, "unit": "GB/s",
+                                    "per_unit": f"dI*2 = {w.dI * 2} B of K^I per cached key (+ q, w, fp32 scores)",
+                                    "units": self.total},
+            "sparse_attn_decode": {"bytes": gather + w.B * w.H * (w.Dqk + w.Dv) * 2, "unit": "GB/s",
+                                   "per_unit": f"Dqk*2 = {w.Dqk * 2} B per selected latent row (+ q, out)",
+                                   "units": w.B * w.k},
+        }
+
+    def host_inputs(self):
+        return {k: v.cpu().pin_memory() for k, v in self.d.items()
+                if isinstance(v, torch.Tensor) and k != "lengths"}
+
+    def load_inputs(self, host):
+        for k, v in host.items():
+            self.d[k].copy_(v, non_blocking=True)
+
+    def result(self):
+        return self.out
+
+
+def time_steps(run, steps, flush):
+    """Per-step and per-kernel device times (ms) over `steps` timed steps."""
+    ev = {"idx": ([], []), "attn": ([], [])}
+    starts, ends = [], []
+    for _ in range(steps):
+        flush.fill_(1)
+        s = PrefillRun._rec()
+        run.step(ev)
+        e = PrefillRun._rec()
+        starts.append(s)
+        ends.append(e)
+    torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    idx_ms = [a.elapsed_time(b) for a, b in zip(*ev["idx"])]
+    # attention segments start where the indexer segment of the same chunk ends
+    attn_ms = [a.elapsed_time(b) for a, b in zip(ev["idx"][1], ev["attn"][1])]
+    return step_ms, idx_ms, attn_ms
+
+
+def time_e2e(run, steps):
+    host = run.host_inputs()
+    res = run.result()
+    res_host = torch.empty(res.shape, dtype=res.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = res.numel() * res.element_size()
+    run.load_inputs(host)
+    run.step()
+    res_host.copy_(res, non_blocking=True)
+    torch.cuda.synchronize()
+    s = PrefillRun._rec()
+    for _ in range(steps):
+        run.load_inputs(host)
+        run.step()
+        res_host.copy_(res, non_blocking=True)
+    e = PrefillRun._rec()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps, h2d, d2h
+
+
+def cpu_baseline(w: W.Workload, budget_s: float = 15.0, run_inputs=None):
+    """The oracle, as it stands, on a seeded sample of the workload's rows."""
+    import oracle as O
+    threads = _blas_threads()
+    if w.kind == "decode":
+        d = run_inputs if run_inputs is not None else W.make_decode_inputs(w, "cpu")
+        cu = d["cu_seqlens"].cpu().numpy()
+        q = d["qI"].cpu().double().numpy()
+        ww = d["w"].cpu().double().numpy()
+        t0 = time.perf_counter()
+        done = 0
+        for b in range(w.B):
+            lo, hi = int(cu[b]), int(cu[b + 1])
+            kc = d["kI_cache"][lo:hi].cpu().double().numpy()
+            s = O.indexer_scores_row(q[b], kc, ww[b])
+            sel = O.causal_topk_row(s, hi - lo - 1, w.k)
+            lat = d["latent_cache"][lo:hi].cpu().double().numpy()
+            O.sparse_attention_row(d["q"][b].cpu().double().numpy(), lat, sel, w.scale, w.Dv)
+            done += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        dt = time.perf_counter() - t0
+        return {"value": done / dt, "unit": METRIC["decode"][1], "cores": threads, "kind": "oracle",
+                "sample": f"{done} of {w.B} sequences of one decode step (float64 numpy)"}
+    d = run_inputs if run_inputs is not None else W.make_prefill_inputs(w, "cpu")
+    rows = W.sample_rows(w, 4096)
+    rng = np.random.default_rng(7)
+    rng.shuffle(rows)
+    t0 = time.perf_counter()
+    done = 0
+    for b, i in rows:
+        _oracle_row(O, w, d, b, i)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": METRIC["prefill"][1], "cores": threads, "kind": "oracle",
+            "sample": f"{done} seeded query rows of B*n={w.B * w.n} (uniform over positions), indexer + top-k + "
+                      f"attention per row, float64 numpy"}
+
+
+def _oracle_row(O, w, d, b, i):
+    if w.fp8:
+        q = O.dequantize(d["qI"][b, i].view(torch.uint8).numpy(), d["q_scale"][b, i].numpy(), 2)
+        k = O.dequantize(d["kI"][b, : i + 1].view(torch.uint8).numpy(), d["k_scale"][b, : i + 1].numpy(), 1)
+    else:
+        q = d["qI"][b, i].double().numpy()
+        k = d["kI"][b, : i + 1].double().numpy()
+    s = O.indexer_scores_row(q, k, d["w"][b, i].double().numpy())
+    sel = O.causal_topk_row(s, i, w.k)
+    lat = d["latent"][b].double().numpy()
+    O.sparse_attention_row(d["q"][b, i].double().numpy(), lat, sel, w.scale, w.Dv)
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def workload_label(w: W.Workload):
+    if w.kind == "decode":
+        return (f"decode B={w.B} L~U[{w.L_min},{w.L_max}] HI={w.HI} dI={w.dI} k={w.k} bf16 K^I cache; "
+                f"attn H={w.H} latent {w.Dqk}/{w.Dv}")
+    dt = "fp8-e4m3 indexer" if w.fp8 else ("bf16 integer-valued indexer" if w.integer_valued else "bf16 indexer")
+    ch = f" in {w.chunk}-query chunks" if w.chunk else ""
+    return (f"prefill B={w.B} n={w.n} HI={w.HI} dI={w.dI} k={w.k} {dt}{ch}; attn H={w.H} latent {w.Dqk}/{w.Dv}")
+
+
+def run_b200(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    from learned_token_indexer_b200.build import build
+    if rank == 0:
+        build()
+    if world > 1:
+        torch.distributed.barrier()
+    w = W.ALL[args.workload]
+    run = DecodeRun(w, dev) if w.kind == "decode" else PrefillRun(w, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        run.step()
+    torch.cuda.synchronize()
+    run.ws_idx.check()
+    run.ws_att.check()
+    sampler = ClockSampler(local)
+    sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    step_ms, idx_ms, attn_ms = time_steps(run, args.steps, flush)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    run.ws_idx.check()
+    run.ws_att.check()
+    ms = float(np.mean(step_ms))
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = time_e2e(run, max(3, min(10, args.steps)))
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * run.rows() / (e2e_ms * 1e-3), "unit": METRIC[w.kind if w.kind == "decode" else "prefill"][1],
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+    peaks, peak_src = load_peaks()
+    work = run.kernel_work()
+    names = list(work.keys())
+    kms = {names[0]: float(np.mean(idx_ms)) / max(1, len(idx_ms) // max(1, args.steps)),
+           names[1]: float(np.mean(attn_ms)) / max(1, len(attn_ms) // max(1, args.steps))}
+    # per launch: each step launches each kernel once per chunk
+    per_step_launches = max(1, len(idx_ms) // max(1, args.steps))
+    kernels = {}
+    for name, wk in work.items():
+        t_launch = float(np.mean(idx_ms if name == names[0] else attn_ms))
+        if "flops" in wk:
+            per_launch = wk["flops"] / per_step_launches
+            peak = peaks["bf16_tflops"] * (2.0 if (w.fp8 and name == names[0]) else 1.0)
+            ach = per_launch / (t_launch * 1e-3) / 1e12
+            bound = "tensor"
+        else:
+            per_launch = wk["bytes"] / per_step_launches
+            peak = peaks["hbm_gbs"]
+            ach = per_launch / (t_launch * 1e-3) / 1e9
+            bound = "hbm"
+        tkey = {"indexer_topk_decode": "indexer_scan", "sparse_attn_decode": "sparse_attn"}.get(name, name)
+        kernels[name] = {"bound": bound, "achieved": round(ach, 2), "peak": peak, "unit": wk["unit"],
+                         "frac": round(ach / peak, 4), "ms_per_launch": round(t_launch, 4),
+                         "traffic": measured_traffic(tkey, w.name),
+                         "algorithmic_per_launch": per_launch, "per_unit": wk["per_unit"]}
+    dom = max(kernels, key=lambda n: kernels[n]["ms_per_launch"])
+    roof = {k: kernels[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{peak_src} ({'fp8 = 2 x measured bf16' if (w.fp8 and roof['bound'] == 'tensor' and dom == names[0]) else 'burst bf16 / copy bandwidth'})"
+    metric, unit = METRIC["decode" if w.kind == "decode" else "prefill"]
+    line = {
+        "metric": metric, "value": world * run.rows() / (ms * 1e-3), "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8-e4m3 indexer / bf16 attention, fp32 accumulate" if w.fp8 else "bf16 in, fp32 accumulate",
+        "data": "synthetic (seeded, HBM-resident)",
+        "config": {"workload": workload_label(w), "global_batch": world * w.B,
+                   "seq_len": w.n if w.kind != "decode" else w.L_max,
+                   "parallelism": f"replicas x{world} (independent batches per GPU)",
+                   "l2": "flushed (256 MiB write) before every timed step, outside the timed events"},
+        "roofline": roof,
+        "kernels": kernels,
+        "gpu_launches": run.launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_budget)
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# reference arm: the oracle on host cores
+# ----------------------------------------------------------------------------
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle as O
+    w = W.ALL[args.workload]
+    metric, unit = METRIC["decode" if w.kind == "decode" else "prefill"]
+    total_budget = args.ref_budget
+    nsteps = args.steps + args.warmup
+    if w.kind == "decode":
+        d = W.make_decode_inputs(w, "cpu")
+        cu = d["cu_seqlens"].numpy()
+        def one(b):
+            lo, hi = int(cu[b]), int(cu[b + 1])
+            s = O.indexer_scores_row(d["qI"][b].double().numpy(), d["kI_cache"][lo:hi].double().numpy(),
+                                     d["w"][b].double().numpy())
+            sel = O.causal_topk_row(s, hi - lo - 1, w.k)
+            O.sparse_attention_row(d["q"][b].double().numpy(), d["latent_cache"][lo:hi].double().numpy(), sel,
+                                   w.scale, w.Dv)
+        units = list(range(w.B))
+        unit_name = "sequences"
+    else:
+        d = W.make_prefill_inputs(w, "cpu")
+        units = W.sample_rows(w, 4096)
+        np.random.default_rng(7).shuffle(units)
+        def one(u):
+            _oracle_row(O, w, d, *u)
+        unit_name = "query rows"
+    t0 = time.perf_counter()
+    one(units[0])
+    per_unit = max(1e-4, time.perf_counter() - t0)
+    per_step = max(1, int(total_budget / nsteps / per_unit))
+    pos = 1
+    def step():
+        nonlocal pos
+        for _ in range(per_step):
+            one(units[pos % len(units)])
+            pos += 1
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = args.steps * per_step / dt
+    threads = _blas_threads()
+    sample = (f"{per_step} seeded {unit_name} per step of B*n={w.B * max(w.n, 1)} "
+              f"({'uniform over positions' if w.kind != 'decode' else 'of one decode step'}), float64 numpy oracle")
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "config": {"workload": workload_label(w)},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="prefill", choices=sorted(W.ALL))
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=90.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_b200(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,171 @@
+/*
+ * dsa.h -- C ABI of libdsa.so, the B200 (sm_100a) implementation of the
+ * DeepSeek Sparse Attention hot path described on the page
+ * "2.2.1 · DSA 与索引器: 先召回 token, 再计算 Sparse MLA":
+ *
+ *   eq. (1)  I[t,s] = sum_j w[t,j] * ReLU(q[t,j] . k[s])        (Lightning Indexer)
+ *   eq. (2)  S_t = TopK({I[t,s] : 0 <= s <= t}, min(k, t+1))     (causal selector)
+ *   eq. (3)  u_t = Attn(h_t, {c_s : s in S_t})                    (sparse attention)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor arguments are DEVICE pointers to contiguous row-major arrays
+ *    owned by the caller.  The library never allocates, frees or synchronises
+ *    (except dsa_read_device_status).  Calls are asynchronous on `stream`
+ *    (a cudaStream_t passed as void*; NULL = legacy default stream).
+ *  - bf16 tensors hold raw bfloat16 bit patterns; FP8 tensors hold E4M3
+ *    ("fn", max 448) codes, one byte each, with one positive fp32 scale per
+ *    token (the dequantised value is code * scale, §2 "quantised indexer key
+ *    cache with scales").
+ *  - Base pointers of the indexer operands (qI, kI) must be 16-byte aligned
+ *    (they are read with TMA); other tensors need their natural alignment.
+ *  - Positions are 0-based.  A query at absolute position t may select keys
+ *    0..t (the current token included).  Index outputs have width k: the
+ *    min(k, t+1) selected positions first, in unspecified order, then -1.
+ *    Equal scores are broken toward the lower position, so the selected set
+ *    is unique.  -0.0 and +0.0 are the same score.
+ *  - Scratch: calls that need scratch memory take a caller-provided device
+ *    workspace of at least the size the matching *_workspace() query returns
+ *    (queries depend only on sizes and on the current device's SM count).
+ *    Every workspace starts with a 256-byte status header: call
+ *    dsa_workspace_init() once after allocating it.  Kernels record the first
+ *    device-side failure there (a bounded wait that gave up, an index outside
+ *    its row); dsa_read_device_status() returns and clears it.  Kernels never
+ *    trap; after such a failure the outputs of that call are unspecified.
+ *  - Host-side argument checks return DSA_ERR_INVALID_ARG / _UNSUPPORTED /
+ *    _WORKSPACE before anything is launched; a failed launch returns
+ *    DSA_ERR_CUDA.  dsa_last_error() gives a message (thread-local).
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARG = 1,   /* bad size, null or misaligned pointer */
+  DSA_ERR_UNSUPPORTED = 2,   /* a size this build has no kernel for */
+  DSA_ERR_WORKSPACE = 3,     /* workspace missing or too small */
+  DSA_ERR_CUDA = 4,          /* a CUDA call or kernel launch failed */
+  DSA_ERR_TIMEOUT = 5,       /* device: a bounded wait gave up */
+  DSA_ERR_DEVICE_CHECK = 6   /* device: an input failed a device-side check */
+} dsa_status;
+
+typedef enum { DSA_BF16 = 0, DSA_FP8_E4M3 = 1 } dsa_dtype;
+
+/* Library version string. */
+const char* dsa_version(void);
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char* dsa_last_error(void);
+/* Name of a status code. */
+const char* dsa_status_string(int status);
+
+/* Time limit of every device-side wait (default 2 s).  Applies to later launches. */
+void dsa_set_wait_timeout_ns(uint64_t ns);
+uint64_t dsa_get_wait_timeout_ns(void);
+
+/* Zero the 256-byte status header at the start of a workspace (async). */
+dsa_status dsa_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+/* Synchronise `stream`, return the device status recorded in `workspace`
+ * (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_CHECK), store its detail word in
+ * *detail if non-NULL, and clear it. */
+dsa_status dsa_read_device_status(void* workspace, void* stream, uint32_t* detail);
+
+/* ------------------------------------------------------------------------
+ * Prefill: fused Lightning Indexer + causal top-k  (eqs. (1) and (2), §1.1;
+ * the fusion of §2: score tiles are filtered as they are produced and merged
+ * into each row's top-k, the score matrix is never written).
+ *
+ * Query rows i = 0..nq-1 of each of B sequences sit at absolute positions
+ * t = q_offset + i; keys 0..kv_len-1 are available (kv_len >= q_offset + nq).
+ *   qI      [B, nq, HI, dI]  bf16 or e4m3 codes
+ *   q_scale [B, nq]          fp32, FP8 only (else NULL): one scale per query token
+ *   kI      [B, kv_len, dI]  bf16 or e4m3 codes
+ *   k_scale [B, kv_len]      fp32, FP8 only (else NULL)
+ *   w       [B, nq, HI]      fp32 head weights (any sign)
+ *   idx_out [B, nq, k]       int32 output (see conventions)
+ *   score_out [B, nq, k]     fp32 output or NULL: the fp32 score of each
+ *                            selected slot, -inf in padding slots.
+ * Supported: HI in {4, 8, 16, 32, 64}; dI <= 128 and a multiple of 8 (bf16)
+ * or 16 (FP8); k >= 1.  Chunked prefill = several calls with increasing
+ * q_offset over the same kI / workspace.
+ * ---------------------------------------------------------------------- */
+size_t dsa_indexer_topk_prefill_workspace(int B, int nq, int kv_len, int HI, int dI, int k, int dtype);
+dsa_status dsa_indexer_topk_prefill(int B, int nq, int q_offset, int kv_len, int HI, int dI, int k, int dtype,
+                                    const void* qI, const float* q_scale, const void* kI, const float* k_scale,
+                                    const float* w, int32_t* idx_out, float* score_out, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Sparse attention, prefill  (eq. (3), §1.1): for each query row and head h,
+ *   z_s = scale * q[h] . c_s over the selected s (slots holding -1 skipped),
+ *   out[h] = softmax_s(z) . c_s[0:Dv],   lse[h] = log sum_s exp(z_s).
+ * The same selected rows serve every head of the row (shared key, §1.1).
+ *   q      [B, nq, H, Dqk]  bf16      latent [B, kv_len, Dqk] bf16 (row c_s)
+ *   idx    [B, nq, k]       int32 positions in [0, kv_len) or -1
+ *   out    [B, nq, H, Dv]   bf16      lse [B, nq, H] fp32 or NULL
+ * A row with no valid slot gives out = 0, lse = -inf.  An index outside
+ * [-1, kv_len) is skipped and recorded as DSA_ERR_DEVICE_CHECK.
+ * Supported: Dqk a multiple of 16, <= 1024; Dv in {64,128,256,512}, Dv <= Dqk.
+ * ---------------------------------------------------------------------- */
+size_t dsa_sparse_attn_workspace(void);
+dsa_status dsa_sparse_attn_prefill(int B, int nq, int kv_len, int H, int Dqk, int Dv, int k, float scale,
+                                   const void* q, const void* latent, const int32_t* idx, void* out, float* lse,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Decode step  (§2: one new query per sequence scans every cached indexer
+ * key; the latent cache is shared by all query heads, MQA form).
+ * Ragged caches: sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1 of
+ * kI_cache / latent_cache; its length L_b includes the new token, which is
+ * the query at local position L_b - 1.  cu_seqlens is a DEVICE int64 array
+ * [B+1]; total_len = cu_seqlens[B] and max_len = max L_b are passed from the
+ * host so nothing has to be read back.
+ *   qI [B, HI, dI], q_scale [B] (FP8) / NULL, w [B, HI],
+ *   kI_cache [total_len, dI], k_scale [total_len] (FP8) / NULL,
+ *   idx_out [B, k] local positions, score_out [B, k] or NULL.
+ * The step's scores (total_len fp32) live in the workspace.
+ * ---------------------------------------------------------------------- */
+size_t dsa_indexer_topk_decode_workspace(int B, int HI, int dI, int k, int dtype, int64_t total_len, int max_len);
+dsa_status dsa_indexer_topk_decode(int B, int HI, int dI, int k, int dtype, const void* qI, const float* q_scale,
+                                   const float* w, const void* kI_cache, const float* k_scale,
+                                   const int64_t* cu_seqlens, int64_t total_len, int max_len, int32_t* idx_out,
+                                   float* score_out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*   q [B, H, Dqk] bf16, latent_cache [total_len, Dqk] bf16, idx [B, k] local
+ *   positions or -1, out [B, H, Dv] bf16, lse [B, H] fp32 or NULL. */
+dsa_status dsa_sparse_attn_decode(int B, int H, int Dqk, int Dv, int k, float scale, const void* q,
+                                  const void* latent_cache, const int64_t* cu_seqlens, int64_t total_len,
+                                  const int32_t* idx, void* out, float* lse, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Debug / test entry points.
+ * dsa_indexer_scores: the dense causal score matrix of eq. (1),
+ *   scores [B, nq, kv_len] fp32, -inf where s > q_offset + i (small n only).
+ * dsa_topk_rows: eq. (2) over materialised rows: row r has row_len[r]
+ *   valid scores (row_len NULL: all ncols) at scores + r*row_stride; the
+ *   first min(k, len) slots get the selected positions (0..len-1), then -1.
+ * dsa_selftest_bounded_wait: runs one kernel whose wait can never complete;
+ *   the wait gives up after timeout_ns and the workspace status becomes
+ *   DSA_ERR_TIMEOUT (exercises the failure path without hanging the GPU).
+ * ---------------------------------------------------------------------- */
+size_t dsa_small_workspace(void);
+dsa_status dsa_indexer_scores(int B, int nq, int q_offset, int kv_len, int HI, int dI, int dtype, const void* qI,
+                              const float* q_scale, const void* kI, const float* k_scale, const float* w,
+                              float* scores, void* workspace, size_t workspace_bytes, void* stream);
+dsa_status dsa_topk_rows(int rows, int ncols, int64_t row_stride, const float* scores, const int32_t* row_len,
+                         int k, int32_t* idx_out, float* val_out, void* workspace, size_t workspace_bytes,
+                         void* stream);
+dsa_status dsa_selftest_bounded_wait(uint64_t timeout_ns, void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

@@ -1,0 +1,254 @@
+"""B200 (sm_100a) DeepSeek Sparse Attention hot path: Python binding.
+
+Every function here marshals torch tensors (device pointers, sizes, the
+current CUDA stream) into one call of libdsa.so (include/dsa.h); all
+arithmetic runs in the library's CUDA kernels.  Torch is used only to
+allocate outputs and workspaces and to provide the stream.
+
+Entry points (page "2.2.1 · DSA 与索引器", §1.1 eqs. (1)-(3), §2 decode):
+    indexer_topk_prefill  fused indexer + causal top-k of a prefill chunk
+    sparse_attn_prefill   sparse attention over the selected latent rows
+    indexer_topk_decode   one decode step of the indexer + top-k (ragged caches)
+    sparse_attn_decode    the decode step's sparse attention (MQA form)
+    indexer_scores, topk_rows, selftest_bounded_wait   debug / test
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+from typing import Optional
+
+import torch
+
+from . import _lib
+
+BF16, FP8_E4M3 = 0, 1
+STATUS = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARG", 2: "DSA_ERR_UNSUPPORTED", 3: "DSA_ERR_WORKSPACE",
+          4: "DSA_ERR_CUDA", 5: "DSA_ERR_TIMEOUT", 6: "DSA_ERR_DEVICE_CHECK"}
+
+
+class DSAError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def lib():
+    return _lib.load()
+
+
+def _check(st: int):
+    if st != 0:
+        raise DSAError(st, lib().dsa_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> C.c_void_p:
+    return C.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype in (torch.float8_e4m3fn, torch.uint8):
+        return FP8_E4M3
+    raise TypeError(f"indexer operands must be bfloat16 or float8_e4m3fn, got {t.dtype}")
+
+
+class Workspace:
+    """A device scratch buffer (256-byte status header + kernel scratch).
+
+    Grows on demand; the header is zeroed once when the buffer is made."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device or "cuda")
+        self.buf: Optional[torch.Tensor] = None
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+            _check(lib().dsa_workspace_init(_ptr(self.buf), self.buf.numel(), _stream(self.device)))
+        return self.buf
+
+    def status(self):
+        """Synchronise and return (status_code, detail); clears the status."""
+        if self.buf is None:
+            return 0, 0
+        d = C.c_uint32(0)
+        st = lib().dsa_read_device_status(_ptr(self.buf), _stream(self.device), C.byref(d))
+        return st, d.value
+
+    def check(self):
+        st, d = self.status()
+        if st != 0:
+            raise DSAError(st, lib().dsa_last_error().decode())
+
+
+_default_ws: dict = {}
+
+
+def _ws(ws: Optional[Workspace], device) -> Workspace:
+    if ws is not None:
+        return ws
+    key = torch.device(device).index if torch.device(device).index is not None else torch.cuda.current_device()
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(torch.device("cuda", key))
+    return _default_ws[key]
+
+
+def version() -> str:
+    return lib().dsa_version().decode()
+
+
+def set_wait_timeout_ns(ns: int):
+    lib().dsa_set_wait_timeout_ns(int(ns))
+
+
+def get_wait_timeout_ns() -> int:
+    return int(lib().dsa_get_wait_timeout_ns())
+
+
+# --------------------------------------------------------------------------
+# Prefill
+# --------------------------------------------------------------------------
+
+def indexer_topk_prefill(qI, kI, w, k: int, q_offset: int = 0, q_scale=None, k_scale=None,
+                         idx_out=None, score_out=None, return_scores: bool = False,
+                         workspace: Optional[Workspace] = None):
+    """Fused eq. (1) + eq. (2) for a prefill chunk.
+
+    qI [B, nq, HI, dI], kI [B, kv_len, dI] (bf16, or e4m3 with q_scale [B, nq]
+    and k_scale [B, kv_len]), w [B, nq, HI] fp32.  Returns idx [B, nq, k]
+    int32 (and scores [B, nq, k] fp32 if asked)."""
+    B, nq, HI, dI = qI.shape
+    kv_len = kI.shape[1]
+    dt = _dtype_code(qI)
+    dev = qI.device
+    if idx_out is None:
+        idx_out = torch.empty((B, nq, k), dtype=torch.int32, device=dev)
+    if return_scores and score_out is None:
+        score_out = torch.empty((B, nq, k), dtype=torch.float32, device=dev)
+    L = lib()
+    need = L.dsa_indexer_topk_prefill_workspace(B, nq, kv_len, HI, dI, k, dt)
+    wsb = _ws(workspace, dev).get(need)
+    _check(L.dsa_indexer_topk_prefill(B, nq, q_offset, kv_len, HI, dI, k, dt, _ptr(qI), _ptr(q_scale), _ptr(kI),
+                                      _ptr(k_scale), _ptr(w), _ptr(idx_out), _ptr(score_out), _ptr(wsb),
+                                      wsb.numel(), _stream(dev)))
+    return (idx_out, score_out) if score_out is not None else idx_out
+
+
+def sparse_attn_prefill(q, latent, idx, dv: int, scale: Optional[float] = None, out=None, lse=None,
+                        return_lse: bool = False, workspace: Optional[Workspace] = None):
+    """Eq. (3): q [B, nq, H, Dqk] bf16, latent [B, kv_len, Dqk] bf16,
+    idx [B, nq, k] int32 -> out [B, nq, H, dv] bf16 (and lse [B, nq, H])."""
+    B, nq, H, Dqk = q.shape
+    kv_len = latent.shape[1]
+    k = idx.shape[-1]
+    scale = Dqk ** -0.5 if scale is None else scale
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, nq, H, dv), dtype=torch.bfloat16, device=dev)
+    if return_lse and lse is None:
+        lse = torch.empty((B, nq, H), dtype=torch.float32, device=dev)
+    L = lib()
+    wsb = _ws(workspace, dev).get(L.dsa_sparse_attn_workspace())
+    _check(L.dsa_sparse_attn_prefill(B, nq, kv_len, H, Dqk, dv, k, float(scale), _ptr(q), _ptr(latent), _ptr(idx),
+                                     _ptr(out), _ptr(lse), _ptr(wsb), wsb.numel(), _stream(dev)))
+    return (out, lse) if lse is not None else out
+
+
+# --------------------------------------------------------------------------
+# Decode
+# --------------------------------------------------------------------------
+
+def indexer_topk_decode(qI, w, kI_cache, cu_seqlens, k: int, total_len: int, max_len: int, q_scale=None,
+                        k_scale=None, idx_out=None, score_out=None, return_scores: bool = False,
+                        workspace: Optional[Workspace] = None):
+    """One decode step of eqs. (1)-(2): qI [B, HI, dI], w [B, HI],
+    kI_cache [total_len, dI], cu_seqlens int64 [B+1] on the device.
+    Returns idx [B, k] of local positions (and scores)."""
+    B, HI, dI = qI.shape
+    dt = _dtype_code(qI)
+    dev = qI.device
+    if idx_out is None:
+        idx_out = torch.empty((B, k), dtype=torch.int32, device=dev)
+    if return_scores and score_out is None:
+        score_out = torch.empty((B, k), dtype=torch.float32, device=dev)
+    L = lib()
+    need = L.dsa_indexer_topk_decode_workspace(B, HI, dI, k, dt, int(total_len), int(max_len))
+    wsb = _ws(workspace, dev).get(need)
+    _check(L.dsa_indexer_topk_decode(B, HI, dI, k, dt, _ptr(qI), _ptr(q_scale), _ptr(w), _ptr(kI_cache),
+                                     _ptr(k_scale), _ptr(cu_seqlens), int(total_len), int(max_len), _ptr(idx_out),
+                                     _ptr(score_out), _ptr(wsb), wsb.numel(), _stream(dev)))
+    return (idx_out, score_out) if score_out is not None else idx_out
+
+
+def sparse_attn_decode(q, latent_cache, cu_seqlens, idx, dv: int, total_len: int, scale: Optional[float] = None,
+                       out=None, lse=None, return_lse: bool = False, workspace: Optional[Workspace] = None):
+    """Eq. (3) for a decode step: q [B, H, Dqk], latent_cache [total_len, Dqk],
+    idx [B, k] local positions -> out [B, H, dv] (and lse [B, H])."""
+    B, H, Dqk = q.shape
+    k = idx.shape[-1]
+    scale = Dqk ** -0.5 if scale is None else scale
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=torch.bfloat16, device=dev)
+    if return_lse and lse is None:
+        lse = torch.empty((B, H), dtype=torch.float32, device=dev)
+    L = lib()
+    wsb = _ws(workspace, dev).get(L.dsa_sparse_attn_workspace())
+    _check(L.dsa_sparse_attn_decode(B, H, Dqk, dv, k, float(scale), _ptr(q), _ptr(latent_cache), _ptr(cu_seqlens),
+                                    int(total_len), _ptr(idx), _ptr(out), _ptr(lse), _ptr(wsb), wsb.numel(),
+                                    _stream(dev)))
+    return (out, lse) if lse is not None else out
+
+
+# --------------------------------------------------------------------------
+# Debug / test
+# --------------------------------------------------------------------------
+
+def indexer_scores(qI, kI, w, q_offset: int = 0, q_scale=None, k_scale=None, out=None,
+                   workspace: Optional[Workspace] = None):
+    """Dense causal scores [B, nq, kv_len] fp32 (-inf beyond the diagonal)."""
+    B, nq, HI, dI = qI.shape
+    kv_len = kI.shape[1]
+    dt = _dtype_code(qI)
+    dev = qI.device
+    if out is None:
+        out = torch.empty((B, nq, kv_len), dtype=torch.float32, device=dev)
+    L = lib()
+    wsb = _ws(workspace, dev).get(L.dsa_small_workspace())
+    _check(L.dsa_indexer_scores(B, nq, q_offset, kv_len, HI, dI, dt, _ptr(qI), _ptr(q_scale), _ptr(kI), _ptr(k_scale),
+                                _ptr(w), _ptr(out), _ptr(wsb), wsb.numel(), _stream(dev)))
+    return out
+
+
+def topk_rows(scores, k: int, row_len=None, idx_out=None, val_out=None, return_values: bool = False,
+              workspace: Optional[Workspace] = None):
+    """Top-k of each row of a [rows, ncols] fp32 matrix (row_len: int32 [rows])."""
+    rows, ncols = scores.shape
+    dev = scores.device
+    if idx_out is None:
+        idx_out = torch.empty((rows, k), dtype=torch.int32, device=dev)
+    if return_values and val_out is None:
+        val_out = torch.empty((rows, k), dtype=torch.float32, device=dev)
+    L = lib()
+    wsb = _ws(workspace, dev).get(L.dsa_small_workspace())
+    _check(L.dsa_topk_rows(rows, ncols, scores.stride(0), _ptr(scores), _ptr(row_len), k, _ptr(idx_out),
+                           _ptr(val_out), _ptr(wsb), wsb.numel(), _stream(dev)))
+    return (idx_out, val_out) if val_out is not None else idx_out
+
+
+def selftest_bounded_wait(timeout_ns: int, workspace: Workspace):
+    L = lib()
+    wsb = workspace.get(L.dsa_small_workspace())
+    _check(L.dsa_selftest_bounded_wait(int(timeout_ns), _ptr(wsb), wsb.numel(), _stream(wsb.device)))

@@ -1,0 +1,429 @@
+// indexer_topk_prefill.cu -- fused Lightning Indexer + causal top-k for a
+// prefill chunk: eqs. (1) and (2) of page "2.2.1 · DSA 与索引器" (§1.1), with
+// the fusion the page's §2 asks for (score tiles are filtered while they are
+// produced and merged into each row's final top-k; the B x n x n score
+// matrix is never written).
+//
+// Work unit: a block of 8 consecutive query tokens of one sequence against
+// all keys 0..t of its last token.  Persistent grid, heavy blocks first, snake
+// order over CTAs.  Per CTA (10 warps):
+//   warp 0      TMA producer: Q of the block (both groups, once), K tiles;
+//   warp 1      tcgen05 MMA issuer, TMEM owner: for each 128-key tile and
+//               each group g of 4 tokens, D_g[128 keys x 4*HI] (+)= K Q_g^T;
+//   warps 2..5  epilogue group 0 (tokens 0..3), warps 6..9 group 1 (4..7):
+//               TMEM -> ReLU * w -> head sum = I[t, s]; causal mask; then
+//               the streaming filter below; after the block's last tile the
+//               exact select (select.cuh) writes idx (and scores).
+// Streaming filter, per token: a 512-bin histogram of accepted scores over a
+// monotone binning of the score (quarter-octaves for 2^-31 <= |x| < 2^31).
+// bin_floor only rises: once at least k accepted entries lie in bins above
+// bin_floor, no later key (higher position) in bin <= bin_floor can enter the
+// top k, so such keys are dropped.  Accepted (key, position) pairs go to a
+// per-(CTA, token slot) candidate buffer in global memory (L2 resident).
+#include "indexer_common.cuh"
+#include "kernels.h"
+#include "select.cuh"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kQB = 8;          // tokens per block
+constexpr int kTA = 4;          // tokens per accumulator group
+constexpr int kPrefillThreads = 320;
+constexpr int kHistBins = 512;  // streaming histogram bins (499 used)
+constexpr uint32_t kLastBin = 498;
+
+__device__ __forceinline__ uint32_t score_bin(uint32_t key) {
+  const uint32_t k11 = key >> 21;
+  if (k11 < 392u) return 0u;                    // x <= -2^31
+  if (k11 < 640u) return 1u + (k11 - 392u);     // -2^31 < x <= -2^-31
+  if (k11 < 1408u) return 249u;                 // |x| < 2^-31 (zeros)
+  if (k11 < 1656u) return 250u + (k11 - 1408u); // 2^-31 <= x < 2^31
+  return kLastBin;                              // x >= 2^31
+}
+
+__device__ __forceinline__ void bin_key_range(uint32_t b, uint32_t& lo, uint32_t& hi) {
+  uint32_t a, z;
+  if (b == 0u) { a = 0u; z = 391u; }
+  else if (b <= 248u) { a = z = 391u + b; }
+  else if (b == 249u) { a = 640u; z = 1407u; }
+  else if (b <= 497u) { a = z = 1408u + (b - 250u); }
+  else { a = 1656u; z = 2047u; }
+  lo = a << 21;
+  hi = (z << 21) | 0x1FFFFFu;
+}
+
+struct Block {
+  int b, t0;      // sequence, first local query row
+  int nvalid;     // valid tokens in the block (<= 8)
+  int nt[2];      // key tiles per group (0 = group empty)
+};
+
+__device__ __forceinline__ bool block_of(const PrefillArgs& a, int r, Block& blk) {
+  // Round r of the snake schedule: CTA c takes item r*G + (c or G-1-c).
+  const int G = gridDim.x;
+  const int c = blockIdx.x;
+  const int item = r * G + ((r & 1) ? (G - 1 - c) : c);
+  const int per_seq = a.nblk - a.first_blk;
+  if (item >= a.B * per_seq) return false;
+  const int j = item / a.B;
+  blk.b = item - j * a.B;
+  const int bi = a.nblk - 1 - j;   // heaviest (last) blocks first
+  blk.t0 = bi * kQB;
+  blk.nvalid = min(kQB, a.nq - blk.t0);
+  for (int g = 0; g < 2; ++g) {
+    const int last = min(blk.t0 + kTA * g + kTA - 1, a.nq - 1);
+    if (blk.t0 + kTA * g >= a.nq) {
+      blk.nt[g] = 0;
+    } else {
+      const int tmax = a.q_offset + last;
+      blk.nt[g] = tmax / kTileKeys + 1;
+    }
+  }
+  return true;
+}
+
+}  // namespace
+
+template <int HI, bool FP8, int KB, int STAGES>
+__global__ void __launch_bounds__(kPrefillThreads, 1)
+    indexer_topk_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                                const __grid_constant__ CUtensorMap tmap_k, const PrefillArgs a) {
+  constexpr int N = kTA * HI;                                 // MMA N per group
+  constexpr int kQGroupBytes = N * KB * kSwizzleBytes;
+  constexpr int kKBytes = kTileKeys * KB * kSwizzleBytes;
+  constexpr uint32_t kTmemCols = (2 * N <= 32) ? 32 : (2 * N <= 64 ? 64 : (2 * N <= 128 ? 128 : (2 * N <= 256 ? 256 : 512)));
+  constexpr uint32_t kIdesc = instr_desc(ElemTraits<FP8>::kFormat, kTileKeys, N);
+  constexpr int kElemsPerBlock = ElemTraits<FP8>::kElemsPerBlock;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = base;
+  uint8_t* sQ = sK + STAGES * kKBytes;
+  float* sW = reinterpret_cast<float*>(sQ + 2 * kQGroupBytes);            // [8][HI]
+  uint32_t* sHist = reinterpret_cast<uint32_t*>(sW + kQB * HI);           // [8][512]
+  uint32_t* sCount = sHist + kQB * kHistBins;                             // [8]
+  uint32_t* sFloor = sCount + kQB;                                        // [8]
+  uint32_t* sBelow = sFloor + kQB;                                        // [8]
+  SelectShared<128>* sSel = reinterpret_cast<SelectShared<128>*>(sBelow + kQB);  // [2]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(sSel + 2) + 7) & ~uintptr_t(7));
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = bars + STAGES;
+  uint64_t* q_full = bars + 2 * STAGES;
+  uint64_t* q_empty = q_full + 1;
+  uint64_t* acc_full = q_empty + 1;   // [2]
+  uint64_t* acc_empty = acc_full + 2; // [2]
+  uint64_t* mma_done = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile uint32_t* abort_flag = tmem_slot + 1;
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&acc_full[g], 1);
+      mbar_init(&acc_empty[g], 4);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0u;
+    mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_k);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl ctl{abort_flag, a.timeout_ns, a.status};
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t kphase = 0, qphase = 0;
+      uint32_t k_last_parity[STAGES];
+      bool k_issued[STAGES];
+      for (int s = 0; s < STAGES; ++s) k_issued[s] = false;
+      bool q_issued = false;
+      uint32_t q_last_parity = 0;
+      bool ok = true;
+      Block blk;
+      for (int r = 0; ok && block_of(a, r, blk); ++r) {
+        if (!(ok = mbar_wait(q_empty, qphase ^ 1u, ctl, 0x1101))) break;
+        mbar_arrive_expect_tx(q_full, 2 * kQGroupBytes);
+        for (int g = 0; g < 2; ++g)
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_2d(sQ + g * kQGroupBytes + kb * N * kSwizzleBytes, &tmap_q, q_full, kb * kElemsPerBlock,
+                        (blk.b * a.nq + blk.t0 + kTA * g) * HI);
+        q_issued = true;
+        q_last_parity = qphase;
+        qphase ^= 1u;
+        const int nt = max(blk.nt[0], blk.nt[1]);
+        for (int t = 0; t < nt; ++t) {
+          if (!(ok = mbar_wait(&k_empty[stage], kphase ^ 1u, ctl, 0x1102))) break;
+          mbar_arrive_expect_tx(&k_full[stage], kKBytes);
+          const int y = blk.b * a.kv_len + t * kTileKeys;
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_2d(sK + stage * kKBytes + kb * kTileKeys * kSwizzleBytes, &tmap_k, &k_full[stage],
+                        kb * kElemsPerBlock, y);
+          k_issued[stage] = true;
+          k_last_parity[stage] = kphase;
+          if (++stage == STAGES) { stage = 0; kphase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        for (int s = 0; s < STAGES; ++s)
+          if (k_issued[s]) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(smem_u32(&k_full[s]), k_last_parity[s]) && globaltimer_ns() - t0 < a.timeout_ns) {
+            }
+          }
+        if (q_issued) {
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(smem_u32(q_full), q_last_parity) && globaltimer_ns() - t0 < a.timeout_ns) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t kphase = 0, qphase = 0, aphase[2] = {0u, 0u};
+      bool ok = true;
+      Block blk;
+      for (int r = 0; ok && block_of(a, r, blk); ++r) {
+        if (!(ok = mbar_wait(q_full, qphase, ctl, 0x1201))) break;
+        qphase ^= 1u;
+        tc_fence_after();
+        const int nt = max(blk.nt[0], blk.nt[1]);
+        for (int t = 0; t < nt && ok; ++t) {
+          if (!(ok = mbar_wait(&k_full[stage], kphase, ctl, 0x1202))) break;
+          tc_fence_after();
+          for (int g = 0; g < 2; ++g) {
+            if (t >= blk.nt[g]) continue;
+            if (!(ok = mbar_wait(&acc_empty[g], aphase[g] ^ 1u, ctl, 0x1203))) break;
+            aphase[g] ^= 1u;
+            tc_fence_after();
+            issue_tile_mma<FP8>(tmem_base + g * N, smem_u32(sK + stage * kKBytes), smem_u32(sQ + g * kQGroupBytes),
+                                N, a.ksteps, kIdesc);
+            tc_commit(&acc_full[g]);
+          }
+          if (!ok) break;
+          tc_commit(&k_empty[stage]);
+          if (++stage == STAGES) { stage = 0; kphase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(q_empty);
+      }
+      tc_commit(mma_done);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(smem_u32(mma_done), 0u) && globaltimer_ns() - t0 < a.timeout_ns) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    // Every thread of a group runs the same sequence of named barriers; a
+    // wait that fails only turns the remaining work into no-ops (no early
+    // exit, so no barrier is ever left short of threads).
+    const uint32_t g = (warp - 2) >> 2;                  // accumulator group 0/1
+    const uint32_t tid = (warp - 2 - 4 * g) * 32 + lane; // 0..127 inside the group
+    const uint32_t bar_id = 2 + g;
+    const uint32_t lane_grp = (warp & 3u) * 32u;
+    const uint32_t key_in_tile = lane_grp + lane;
+    SelectShared<128>& sel = sSel[g];
+    uint32_t aphase = 0;
+    bool ok = true;
+    Block blk;
+    for (int r = 0; block_of(a, r, blk); ++r) {
+      named_bar_sync(bar_id, 128);
+      // per-block state of this group's 4 tokens
+      int tok_t[kTA];
+      bool tok_valid[kTA];
+#pragma unroll
+      for (int j = 0; j < kTA; ++j) {
+        const int li = blk.t0 + kTA * (int)g + j;
+        tok_valid[j] = li < a.nq;
+        tok_t[j] = a.q_offset + li;
+      }
+      for (int i = (int)tid; i < kTA * kHistBins; i += 128) sHist[(kTA * g) * kHistBins + i] = 0u;
+      if (tid < (uint32_t)kTA) {
+        sCount[kTA * g + tid] = 0u;
+        sFloor[kTA * g + tid] = 0u;
+        sBelow[kTA * g + tid] = 0u;
+      }
+      for (int i = (int)tid; i < kTA * HI; i += 128) {
+        const int j = i / HI, h = i - j * HI;
+        const int li = blk.t0 + kTA * (int)g + j;
+        float wv = 0.0f;
+        if (li < a.nq) {
+          const int64_t row = (int64_t)blk.b * a.nq + li;
+          wv = a.w[row * HI + h];
+          if (FP8) wv *= a.q_scale[row];
+        }
+        sW[(kTA * g + j) * HI + h] = wv;
+      }
+      named_bar_sync(bar_id, 128);
+      const int nt = blk.nt[g];
+      uint2* cand_base = a.cand + ((int64_t)blockIdx.x * kQB + kTA * g) * a.cand_cap;
+      for (int t = 0; t < nt; ++t) {
+        bool got = ok && mbar_wait(&acc_full[g], aphase, ctl, 0x1301);
+        ok = __all_sync(0xffffffffu, got);
+        aphase ^= 1u;
+        const int s = t * kTileKeys + (int)key_in_tile;
+        float score[kTA];
+        if (ok) {
+          tc_fence_after();
+          float ks = 1.0f;
+          if (FP8) ks = (s < a.kv_len) ? a.k_scale[(int64_t)blk.b * a.kv_len + s] : 0.0f;
+#pragma unroll
+          for (int j = 0; j < kTA; ++j) {
+            uint32_t rr[HI];
+            tmem_load_heads<HI>(tmem_base + (lane_grp << 16) + g * N + j * HI, rr);
+            tmem_wait_ld();
+            score[j] = relu_weighted_head_sum<HI>(rr, sW + (kTA * g + j) * HI);
+            if (FP8) score[j] *= ks;
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[g]);
+        }
+        named_bar_sync(bar_id, 128);     // previous tile's floor update is visible
+        if (ok) {
+#pragma unroll
+          for (int j = 0; j < kTA; ++j) {
+            const uint32_t key = float_to_key(score[j]);
+            const uint32_t bin = score_bin(key);
+            const bool acc = tok_valid[j] && s <= tok_t[j] && bin >= sFloor[kTA * g + j];
+            const uint32_t mask = __ballot_sync(0xffffffffu, acc);
+            if (mask) {
+              uint32_t slot0 = 0;
+              if (lane == 0) slot0 = atomicAdd(&sCount[kTA * g + j], (uint32_t)__popc(mask));
+              slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+              if (acc) {
+                const uint32_t slot = slot0 + __popc(mask & ((1u << lane) - 1u));
+                cand_base[(int64_t)j * a.cand_cap + slot] = make_uint2(key, (uint32_t)s);
+                atomicAdd(&sHist[(kTA * g + j) * kHistBins + bin], 1u);
+              }
+            }
+          }
+        }
+        named_bar_sync(bar_id, 128);     // this tile's appends are complete
+        if (ok && tid < (uint32_t)kTA) {
+          const uint32_t* h = sHist + (kTA * g + tid) * kHistBins;
+          const uint32_t c = sCount[kTA * g + tid];
+          uint32_t fl = sFloor[kTA * g + tid], bl = sBelow[kTA * g + tid];
+          while (fl < kLastBin && c - bl - h[fl] >= (uint32_t)a.k) {
+            bl += h[fl];
+            ++fl;
+          }
+          sFloor[kTA * g + tid] = fl;
+          sBelow[kTA * g + tid] = bl;
+        }
+      }
+      named_bar_sync(bar_id, 128);
+      if (tid == 0) sel.aborted = *abort_flag;
+      named_bar_sync(bar_id, 128);
+      if (sel.aborted) continue;   // group-uniform: nothing below is valid
+      // ---- exact select of each token's top min(k, t+1)
+      for (int j = 0; j < kTA; ++j) {
+        if (!tok_valid[j] || nt == 0) continue;
+        const int kk = min(a.k, tok_t[j] + 1);
+        const int m = (int)sCount[kTA * g + j];
+        uint32_t* hist = sHist + (kTA * g + j) * kHistBins;
+        const uint2* buf = cand_base + (int64_t)j * a.cand_cap;
+        auto get = [buf](int i, uint32_t& key, uint32_t& pos) {
+          const uint2 e = buf[i];
+          key = e.x;
+          pos = e.y;
+        };
+        group_find<128>(hist, kHistBins, (uint32_t)kk, true, sel, tid, bar_id);
+        const uint32_t b0 = sel.found_bin;
+        const uint32_t need = (uint32_t)kk - sel.found_beyond;
+        const uint32_t cnt = hist[b0];
+        named_bar_sync(bar_id, 128);   // hist of this token becomes scratch
+        SelectResult res;
+        bin_key_range(b0, res.lo, res.hi);
+        res.key_all_in = 1;
+        res.pos_hi = 0;
+        if (need != cnt)
+          res = group_refine<128, kHistBins>(get, m, res.lo, res.hi, need, (uint32_t)tok_t[j], hist, sel, tid,
+                                             bar_id);
+        const int64_t row = (int64_t)blk.b * a.nq + blk.t0 + kTA * g + j;
+        group_emit<128>(get, m, res, kk, a.k, a.idx_out + row * a.k,
+                        a.score_out ? a.score_out + row * a.k : nullptr, sel, tid, bar_id, a.status);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+template <int HI, bool FP8, int KB>
+struct PrefillConfig {
+  static constexpr int N = kTA * HI;
+  static constexpr int kQBytes = 2 * N * KB * kSwizzleBytes;
+  static constexpr int kKBytes = kTileKeys * KB * kSwizzleBytes;
+  static constexpr int kFixed = 1024 /*align*/ + kQBytes + kQB * HI * 4 + kQB * kHistBins * 4 + 3 * kQB * 4 +
+                                2 * (int)sizeof(SelectShared<128>) + 8 + 16 * 8 + 16;
+  static constexpr int kBudget = 227 * 1024;
+  static constexpr int kStagesFit = (kBudget - kFixed) / kKBytes;
+  static constexpr int STAGES = kStagesFit > 6 ? 6 : kStagesFit;
+  static_assert(STAGES >= 2, "not enough shared memory for two K stages");
+  static constexpr int kSmem = kFixed + STAGES * kKBytes + 2 * STAGES * 8;
+};
+
+template <int HI, bool FP8, int KB>
+static cudaError_t launch_prefill_t(const CUtensorMap& tq, const CUtensorMap& tk, const PrefillArgs& a, int grid,
+                                    cudaStream_t stream) {
+  using C = PrefillConfig<HI, FP8, KB>;
+  auto kern = indexer_topk_prefill_kernel<HI, FP8, KB, C::STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kPrefillThreads, C::kSmem, stream>>>(tq, tk, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_indexer_topk_prefill(int HI, bool fp8, int kblocks, const CUtensorMap& tq,
+                                        const CUtensorMap& tk, const PrefillArgs& a, int grid, cudaStream_t stream) {
+#define DSA_PF_CASE(H)                                                          \
+  case H:                                                                       \
+    if (fp8) return launch_prefill_t<H, true, 1>(tq, tk, a, grid, stream);      \
+    if (kblocks == 1) return launch_prefill_t<H, false, 1>(tq, tk, a, grid, stream); \
+    return launch_prefill_t<H, false, 2>(tq, tk, a, grid, stream);
+  switch (HI) {
+    DSA_PF_CASE(4)
+    DSA_PF_CASE(8)
+    DSA_PF_CASE(16)
+    DSA_PF_CASE(32)
+    DSA_PF_CASE(64)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef DSA_PF_CASE
+}
+
+int prefill_block_tokens() { return kQB; }
+
+}  // namespace dsa

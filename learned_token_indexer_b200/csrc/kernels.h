@@ -1,0 +1,87 @@
+// kernels.h -- internal interface between the C ABI (api.cu) and the kernels.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace dsa {
+
+struct DeviceStatus;
+
+// Dense score rows (indexer_scan.cu).
+struct ScanArgs {
+  int mode;                    // 0: prefill rows (b, i); 1: ragged decode rows
+  int rows;                    // prefill B*nq; decode B
+  int nq, q_offset, kv_len;    // prefill geometry
+  const int64_t* cu_seqlens;   // decode: [rows + 1]
+  int ksteps;                  // 32-byte MMA K steps holding data
+  int chunk_tiles;             // key tiles per work item
+  int max_chunks;              // work items per row (upper bound)
+  const float* w;              // [rows, HI]
+  const float* q_scale;        // [rows] (FP8) or null
+  const float* k_scale;        // [key rows] (FP8) or null
+  float* out;                  // prefill [rows, kv_len]; decode [sum L]
+  DeviceStatus* status;
+  uint64_t timeout_ns;
+};
+
+// Fused prefill indexer + top-k (indexer_topk_prefill.cu).
+struct PrefillArgs {
+  int B, nq, q_offset, kv_len, k;
+  int ksteps;
+  int nblk;                    // 8-token blocks per sequence
+  int first_blk;               // blocks below this one need no scoring
+  const float* w;              // [B, nq, HI]
+  const float* q_scale;        // [B, nq] (FP8) or null
+  const float* k_scale;        // [B, kv_len] (FP8) or null
+  int32_t* idx_out;            // [B, nq, k]
+  float* score_out;            // [B, nq, k] or null
+  uint2* cand;                 // [grid * 8, cand_cap] candidate (key, pos) buffers
+  int64_t cand_cap;
+  DeviceStatus* status;
+  uint64_t timeout_ns;
+};
+
+// Row-wise top-k over materialised scores (topk.cu).
+struct TopkRowsArgs {
+  int rows, k;
+  const float* scores;
+  int64_t row_stride;          // used when cu_seqlens == null
+  const int32_t* row_len;      // [rows] or null (then every row has ncols)
+  int ncols;
+  const int64_t* cu_seqlens;   // ragged rows: row r = scores[cu[r] .. cu[r+1])
+  int32_t* idx_out;            // [rows, k]
+  float* val_out;              // [rows, k] or null
+  DeviceStatus* status;
+};
+
+// Sparse attention over selected latent rows (sparse_attn.cu).
+struct AttnArgs {
+  int rows;                    // query rows (prefill B*nq, decode B)
+  int H, Dqk, Dv, k;
+  float scale_log2;            // softmax scale * log2(e)
+  float scale;
+  const uint16_t* q;           // [rows, H, Dqk] bf16
+  const uint16_t* latent;      // prefill [B, kv_len, Dqk]; decode [sum L, Dqk]
+  const int32_t* idx;          // [rows, k]
+  int mode;                    // 0 prefill (row r -> b = r / nq), 1 decode (cu_seqlens)
+  int nq, kv_len;
+  const int64_t* cu_seqlens;
+  uint16_t* out;               // [rows, H, Dv] bf16
+  float* lse;                  // [rows, H] or null
+  DeviceStatus* status;
+};
+
+cudaError_t launch_indexer_scan(int HI, bool fp8, int kblocks, const CUtensorMap& tq, const CUtensorMap& tk,
+                                const ScanArgs& a, int grid, cudaStream_t stream);
+cudaError_t launch_indexer_topk_prefill(int HI, bool fp8, int kblocks, const CUtensorMap& tq,
+                                        const CUtensorMap& tk, const PrefillArgs& a, int grid, cudaStream_t stream);
+int prefill_block_tokens();
+cudaError_t launch_topk_rows(const TopkRowsArgs& a, cudaStream_t stream);
+cudaError_t launch_fill_trivial_rows(int B, int nq, int q_offset, int rows_per_seq, int k, int32_t* idx,
+                                     cudaStream_t stream);
+cudaError_t launch_fill_f32(float* p, int64_t n, float v, cudaStream_t stream);
+cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_wait_selftest(DeviceStatus* status, uint64_t timeout_ns, cudaStream_t stream);
+
+}  // namespace dsa

@@ -1,0 +1,198 @@
+// select.cuh -- exact top-k selection of one row by radix refinement, done by
+// a group of NT threads that share a histogram in shared memory.
+//
+// Eq. (2) of page "2.2.1 · DSA 与索引器" (§1.1): S_t = TopK({I[t,s]}, min(k, t+1)).
+// Entries are (key, pos) with key = order-preserving uint32 image of the
+// score (-0.0 folded into +0.0) and pos the key position; the order is key
+// descending, then position ascending (ties go to the lower position), so the
+// selected set is unique.  The page (§2, top-k paragraph) names radix top-k as
+// the usual way to avoid an O(t log t) sort; this is such a select:
+//
+//   1. keep an interval [lo, hi] of keys known to contain the cut-off key, and
+//      `need` = how many entries inside the interval still have to be taken;
+//   2. histogram the entries inside the interval by their next digit, find
+//      the digit bin where the running count (from the top) reaches `need`,
+//      and shrink the interval to that bin; stop early when the whole bin is
+//      taken;
+//   3. if the interval shrinks to one key with more entries than `need`,
+//      refine the same way over positions (from the bottom: lowest first);
+//   4. one output pass writes every selected entry in unspecified slot order.
+#pragma once
+#include "sm100.cuh"
+
+namespace dsa {
+
+struct SelectResult {
+  uint32_t lo, hi;        // key interval of the cut-off
+  uint32_t key_all_in;    // 1: every entry with key >= lo is selected
+  uint32_t pos_hi;        // else: key == lo entries with pos <= pos_hi are selected
+};
+
+// Shared scratch of one selecting group.
+template <int NT>
+struct SelectShared {
+  uint32_t warp_sum[NT / 32];
+  uint32_t found_bin;
+  uint32_t found_beyond;
+  uint32_t out_count;
+  uint32_t aborted;
+};
+
+// Find the bin where the running count over `nbins` bins, traversed from the
+// top (from_top) or from the bottom, first reaches `need` (1 <= need <= total).
+// Result: sh.found_bin, sh.found_beyond = count strictly before it in
+// traversal order.  All NT threads call it; it ends with a barrier.
+template <int NT>
+__device__ __forceinline__ void group_find(const uint32_t* hist, int nbins, uint32_t need, bool from_top,
+                                           SelectShared<NT>& sh, uint32_t tid, uint32_t bar_id) {
+  const int per = (nbins + NT - 1) / NT;
+  const int i0 = (int)tid * per;
+  uint32_t local = 0;
+  for (int i = i0; i < i0 + per && i < nbins; ++i) local += hist[from_top ? nbins - 1 - i : i];
+  const uint32_t lane = tid & 31u, w = tid >> 5;
+  uint32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= (uint32_t)o) incl += v;
+  }
+  if (lane == 31) sh.warp_sum[w] = incl;
+  named_bar_sync(bar_id, NT);
+  uint32_t before = incl - local;
+  for (uint32_t j = 0; j < w; ++j) before += sh.warp_sum[j];
+  if (before < need && need <= before + local) {
+    uint32_t run = before;
+    for (int i = i0; i < i0 + per && i < nbins; ++i) {
+      const int b = from_top ? nbins - 1 - i : i;
+      const uint32_t h = hist[b];
+      if (run + h >= need) {
+        sh.found_bin = (uint32_t)b;
+        sh.found_beyond = run;
+        break;
+      }
+      run += h;
+    }
+  }
+  named_bar_sync(bar_id, NT);
+}
+
+// Refine a cut-off inside [lo, hi] (need >= 1 entries to take there, entries
+// above hi already counted).  `get(i, key, pos)` reads entry i < m.
+// `hist` is NBINS uint32 of shared scratch owned by the group.
+template <int NT, int NBINS, typename Get>
+__device__ SelectResult group_refine(Get get, int m, uint32_t lo, uint32_t hi, uint32_t need, uint32_t pos_max,
+                                     uint32_t* hist, SelectShared<NT>& sh, uint32_t tid, uint32_t bar_id) {
+  SelectResult r;
+  r.key_all_in = 0;
+  r.pos_hi = 0;
+  bool done = false;
+  while (!done && lo < hi) {
+    int s = 0;
+    while (((hi >> s) - (lo >> s)) >= (uint32_t)NBINS) ++s;
+    const uint32_t base = lo >> s;
+    const int nb = (int)((hi >> s) - base) + 1;
+    for (int i = (int)tid; i < nb; i += NT) hist[i] = 0u;
+    named_bar_sync(bar_id, NT);
+    for (int i = (int)tid; i < m; i += NT) {
+      uint32_t key, pos;
+      get(i, key, pos);
+      if (key >= lo && key <= hi) atomicAdd(&hist[(key >> s) - base], 1u);
+    }
+    named_bar_sync(bar_id, NT);
+    group_find<NT>(hist, nb, need, true, sh, tid, bar_id);
+    const uint32_t d = sh.found_bin;
+    const uint32_t cnt = hist[d];
+    need -= sh.found_beyond;
+    const uint64_t nlo = (uint64_t)(base + d) << s;
+    const uint64_t nhi = (((uint64_t)(base + d) + 1) << s) - 1;
+    lo = nlo > lo ? (uint32_t)nlo : lo;
+    hi = nhi < hi ? (uint32_t)nhi : hi;
+    if (need == cnt) done = true;
+    named_bar_sync(bar_id, NT);
+  }
+  r.lo = lo;
+  r.hi = hi;
+  if (done) {
+    r.key_all_in = 1;
+    return r;
+  }
+  // One key (lo == hi) holds more entries than needed: take the lowest positions.
+  uint32_t plo = 0, phi = pos_max;
+  bool pdone = false;
+  while (!pdone) {
+    int s = 0;
+    while (((phi >> s) - (plo >> s)) >= (uint32_t)NBINS) ++s;
+    const uint32_t base = plo >> s;
+    const int nb = (int)((phi >> s) - base) + 1;
+    for (int i = (int)tid; i < nb; i += NT) hist[i] = 0u;
+    named_bar_sync(bar_id, NT);
+    for (int i = (int)tid; i < m; i += NT) {
+      uint32_t key, pos;
+      get(i, key, pos);
+      if (key == lo && pos >= plo && pos <= phi) atomicAdd(&hist[(pos >> s) - base], 1u);
+    }
+    named_bar_sync(bar_id, NT);
+    group_find<NT>(hist, nb, need, false, sh, tid, bar_id);
+    const uint32_t d = sh.found_bin;
+    const uint32_t cnt = hist[d];
+    need -= sh.found_beyond;
+    const uint64_t nlo = (uint64_t)(base + d) << s;
+    const uint64_t nhi = (((uint64_t)(base + d) + 1) << s) - 1;
+    plo = nlo > plo ? (uint32_t)nlo : plo;
+    phi = nhi < phi ? (uint32_t)nhi : phi;
+    if (need == cnt) pdone = true;
+    named_bar_sync(bar_id, NT);
+  }
+  r.pos_hi = phi;
+  return r;
+}
+
+__device__ __forceinline__ bool selected(const SelectResult& r, uint32_t key, uint32_t pos) {
+  if (key > r.hi) return true;
+  if (key < r.lo) return false;
+  return r.key_all_in || pos <= r.pos_hi;
+}
+
+// Write the selected entries (exactly kk of them) to idx_row[0..kk) in
+// unspecified order, scores too if score_row != nullptr, then pad [kk, k)
+// with -1 / -inf.
+template <int NT, typename Get>
+__device__ void group_emit(Get get, int m, const SelectResult& r, int kk, int k, int32_t* idx_row,
+                           float* score_row, SelectShared<NT>& sh, uint32_t tid, uint32_t bar_id,
+                           DeviceStatus* status) {
+  if (tid == 0) sh.out_count = 0;
+  named_bar_sync(bar_id, NT);
+  const uint32_t lane = tid & 31u;
+  for (int i0 = 0; i0 < m; i0 += NT) {
+    const int i = i0 + (int)tid;
+    uint32_t key = 0, pos = 0;
+    bool sel = false;
+    if (i < m) {
+      get(i, key, pos);
+      sel = selected(r, key, pos);
+    }
+    const uint32_t mask = __ballot_sync(0xffffffffu, sel);
+    uint32_t base = 0;
+    if (lane == 0 && mask) base = atomicAdd(&sh.out_count, (uint32_t)__popc(mask));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    if (sel) {
+      const uint32_t slot = base + __popc(mask & ((1u << lane) - 1u));
+      if (slot < (uint32_t)kk) {
+        idx_row[slot] = (int32_t)pos;
+        if (score_row) score_row[slot] = key_to_float(key);
+      }
+    }
+  }
+  named_bar_sync(bar_id, NT);
+  // A selection that does not produce exactly kk entries is a library bug:
+  // report it and leave no stale slot behind.
+  const int got = (int)sh.out_count;
+  if (got != kk && tid == 0) report_status(status, kStatusDeviceCheck, 0x5e1ec7u);
+  for (int j = (got < kk ? got : kk) + (int)tid; j < k; j += NT) {
+    idx_row[j] = -1;
+    if (score_row) score_row[j] = -__int_as_float(0x7f800000);
+  }
+  named_bar_sync(bar_id, NT);
+}
+
+}  // namespace dsa

@@ -1,0 +1,117 @@
+"""The C-ABI library: it loads, exports every function include/dsa.h declares,
+and its host-side argument checks reject bad calls before touching a GPU."""
+
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import learned_token_indexer_b200 as dsa
+from learned_token_indexer_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(dsa_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from learned_token_indexer_b200.build import build
+    build()
+    return _lib.load()
+
+
+def test_header_declares_the_hot_path():
+    names = _declared_functions()
+    for required in ("dsa_indexer_topk_prefill", "dsa_sparse_attn_prefill", "dsa_indexer_topk_decode",
+                     "dsa_sparse_attn_decode", "dsa_topk_rows", "dsa_indexer_scores"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding has no signature for {name}"
+
+
+def test_no_torch_in_the_boundary():
+    text = open(HEADER).read()
+    assert "torch" not in text.lower().replace("no torch", "")
+    assert "at::" not in text
+
+
+def test_version_and_status_strings(lib):
+    assert b"sm_100a" in lib.dsa_version()
+    assert lib.dsa_status_string(5) == b"DSA_ERR_TIMEOUT"
+    assert lib.dsa_status_string(99) == b"unknown dsa_status"
+
+
+def test_timeout_setting_roundtrip(lib):
+    old = lib.dsa_get_wait_timeout_ns()
+    lib.dsa_set_wait_timeout_ns(12345)
+    assert lib.dsa_get_wait_timeout_ns() == 12345
+    lib.dsa_set_wait_timeout_ns(old)
+
+
+def _prefill(lib, **kw):
+    a = dict(B=1, nq=16, q_offset=0, kv_len=16, HI=64, dI=128, k=8, dtype=0, q=16, qs=None, kI=16, ks=None, w=16,
+             idx=16, sc=None, ws=256, wsb=1 << 30)
+    a.update(kw)
+    p = lambda v: None if v is None else C.c_void_p(v)
+    return lib.dsa_indexer_topk_prefill(a["B"], a["nq"], a["q_offset"], a["kv_len"], a["HI"], a["dI"], a["k"],
+                                        a["dtype"], p(a["q"]), p(a["qs"]), p(a["kI"]), p(a["ks"]), p(a["w"]),
+                                        p(a["idx"]), p(a["sc"]), p(a["ws"]), a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(HI=3), 2),                 # unsupported head count
+    (dict(HI=128), 2),
+    (dict(dI=100), 2),               # not a multiple of 8
+    (dict(dI=136), 2),
+    (dict(dtype=1, dI=120), 2),      # FP8 needs a multiple of 16
+    (dict(dtype=7), 1),
+    (dict(k=0), 1),
+    (dict(q_offset=4, nq=16, kv_len=16), 1),   # rows past the keys
+    (dict(q=None), 1),
+    (dict(q=24), 1),                 # misaligned TMA operand
+    (dict(dtype=1, qs=None, ks=None), 1),      # FP8 without scales
+    (dict(ws=None), 3),
+    (dict(ws=512 + 16), 3),          # misaligned workspace
+    (dict(wsb=64), 3),               # too small
+])
+def test_prefill_argument_checks(lib, kw, status):
+    assert _prefill(lib, **kw) == status
+    assert lib.dsa_last_error()
+
+
+def test_attention_argument_checks(lib):
+    f = lib.dsa_sparse_attn_prefill
+    v = C.c_void_p(256)
+    assert f(1, 4, 16, 16, 576, 500, 8, 0.1, v, v, v, v, None, v, 256, None) == 2     # Dv
+    assert f(1, 4, 16, 16, 72, 64, 8, 0.1, v, v, v, v, None, v, 256, None) == 2      # Dqk % 16
+    assert f(1, 4, 16, 16, 576, 512, 0, 0.1, v, v, v, v, None, v, 256, None) == 1    # k
+    assert f(1, 4, 16, 16, 576, 512, 8, float("nan"), v, v, v, v, None, v, 256, None) == 1
+    assert f(1, 4, 16, 16, 576, 512, 8, 0.1, v, v, v, v, None, v, 8, None) == 3     # workspace
+
+
+def test_workspace_sizes(lib):
+    small = lib.dsa_small_workspace()
+    assert small == 256
+    pf = lib.dsa_indexer_topk_prefill_workspace(1, 8192, 8192, 64, 128, 2048, 0)
+    assert pf > 256 and (pf - 256) % (8 * 8192 * 8) == 0
+    dec = lib.dsa_indexer_topk_decode_workspace(64, 64, 128, 2048, 0, 1000, 100)
+    assert dec >= 256 + 4000
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        _lib.load()

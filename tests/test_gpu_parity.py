@@ -1,0 +1,392 @@
+"""GPU parity: the CUDA path (called through the C ABI) against the CPU oracle
+on the same seeded inputs.
+
+Integer-valued indexer inputs give exact fp32 scores, so there indices must
+match the oracle bit for bit (ties to the lower position on both sides).
+Float inputs use the tolerance-aware selection check (tests/checks.py) and
+attention uses |gpu - oracle| <= 2e-2 + 1e-2 |oracle| (bf16), 5e-2 for the
+FP8 workload, with the oracle's eq. (3) run on the GPU's own indices.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import learned_token_indexer_b200 as dsa
+import oracle as O
+from learned_token_indexer_b200 import workloads as W
+from tests import checks
+from tests.gpu_util import host_f64, indexer_host_inputs
+
+pytestmark = pytest.mark.gpu
+
+ATOL, RTOL = 2e-2, 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from learned_token_indexer_b200.build import build
+    build()
+    torch.cuda.init()
+    yield
+
+
+def _ws():
+    return dsa.Workspace("cuda")
+
+
+def _no_device_errors(ws):
+    st, detail = ws.status()
+    assert st == 0, f"device status {dsa.STATUS.get(st)} detail 0x{detail:x}"
+
+
+# --------------------------------------------------------------------------
+# bounded waits and device checks
+# --------------------------------------------------------------------------
+
+def test_bounded_wait_times_out_with_status():
+    ws = _ws()
+    dsa.selftest_bounded_wait(2_000_000, ws)          # 2 ms
+    st, detail = ws.status()
+    assert st == 5 and detail == 0x7E57
+    _no_device_errors(ws)                             # status was cleared
+    x = torch.ones(4, device="cuda")                  # the context still works
+    assert float(x.sum()) == 4.0
+
+
+# --------------------------------------------------------------------------
+# eq. (1): dense scores through the tcgen05 scan kernel
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("HI,dI", [(4, 32), (8, 64), (16, 128), (32, 96), (64, 128), (64, 64)])
+def test_indexer_scores_integer_exact(HI, dI):
+    w = W.scaled(W.TINY, B=2, n=300, HI=HI, dI=dI, qk_int_max=3, w_den=8, seed=11 + HI)
+    d = W.make_prefill_inputs(w, "cuda", with_attention=False)
+    ws = _ws()
+    got = dsa.indexer_scores(d["qI"], d["kI"], d["w"], workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    q, k, wt = indexer_host_inputs(d)
+    ref = O.indexer_scores(q, k, wt)
+    assert np.array_equal(got.cpu().double().numpy(), ref)
+
+
+def test_indexer_scores_with_offset_and_fp8():
+    w = W.scaled(W.PREFILL_FP8, B=2, n=384, seed=5)
+    d = W.make_prefill_inputs(w, "cuda", with_attention=False)
+    ws = _ws()
+    got = dsa.indexer_scores(d["qI"][:, 128:].contiguous(), d["kI"], d["w"][:, 128:].contiguous(), q_offset=128,
+                             q_scale=d["q_scale"][:, 128:].contiguous(), k_scale=d["k_scale"], workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    q, k, wt = indexer_host_inputs(d)
+    ref = O.indexer_scores(q[:, 128:], k, wt[:, 128:], q_offset=128)
+    g = got.cpu().double().numpy()
+    assert np.array_equal(np.isneginf(g), np.isneginf(ref))
+    fin = np.isfinite(ref)
+    scale = np.abs(ref[fin]).max()
+    assert np.max(np.abs(g[fin] - ref[fin])) <= 1e-5 * scale
+
+
+# --------------------------------------------------------------------------
+# eq. (2): standalone row top-k
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("k", [1, 7, 64, 2048])
+def test_topk_rows_exact_with_ties(k):
+    g = torch.Generator().manual_seed(k)
+    rows, ncols = 33, 5000
+    s = torch.randint(-40, 40, (rows, ncols), generator=g).float() / 4     # many ties
+    s[3] = 0.0
+    s[4, ::2] = -0.0                                                       # -0 == +0
+    s[5] = torch.randn(ncols, generator=g)
+    lens = torch.randint(0, ncols + 1, (rows,), generator=g).int()
+    lens[0], lens[1], lens[2] = 0, 1, ncols
+    ws = _ws()
+    idx, val = dsa.topk_rows(s.cuda(), k, row_len=lens.cuda(), return_values=True, workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    idx, val = idx.cpu().numpy(), val.cpu().numpy()
+    for r in range(rows):
+        L = int(lens[r])
+        if L == 0:
+            assert np.all(idx[r] == -1)
+            continue
+        ref = O.causal_topk_row(s[r, :L].double().numpy(), L - 1, k)
+        errs = checks.topk_exact_errors(idx[r], ref, L - 1, k)
+        assert not errs, errs
+        m = min(k, L)
+        assert np.array_equal(val[r, :m], s[r, idx[r, :m]].numpy() + 0.0)
+
+
+# --------------------------------------------------------------------------
+# eqs. (1)+(2) fused, prefill
+# --------------------------------------------------------------------------
+
+def _prefill_exact(w, q_offset=0, nq=None, chunk=None, rows=None):
+    d = W.make_prefill_inputs(w, "cuda", with_attention=False)
+    n = w.n
+    ws = _ws()
+    if chunk is None:
+        idx = dsa.indexer_topk_prefill(d["qI"], d["kI"], d["w"], w.k, workspace=ws)
+    else:
+        idx = torch.empty((w.B, n, w.k), dtype=torch.int32, device="cuda")
+        for c0 in range(0, n, chunk):
+            c1 = min(n, c0 + chunk)
+            dsa.indexer_topk_prefill(d["qI"][:, c0:c1], d["kI"], d["w"][:, c0:c1], w.k, q_offset=c0,
+                                     idx_out=idx[:, c0:c1], workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    q, k, wt = indexer_host_inputs(d)
+    todo = rows if rows is not None else [(b, i) for b in range(w.B) for i in range(n)]
+    ref = O.indexer_topk(q, k, wt, w.k, rows=todo)
+    idx = idx.cpu().numpy()
+    bad = []
+    for b, i in todo:
+        bad += checks.topk_exact_errors(idx[b, i], ref[b, i], i, w.k)
+    assert not bad, bad[:5]
+
+
+def test_prefill_tiny_exact():
+    _prefill_exact(W.TINY)
+
+
+@pytest.mark.parametrize("HI,dI,n,k", [(64, 128, 1000, 100), (16, 64, 777, 33), (8, 32, 530, 300),
+                                       (64, 128, 1100, 1)])
+def test_prefill_integer_exact_ragged(HI, dI, n, k):
+    w = W.scaled(W.PREFILL, B=2, n=n, HI=HI, dI=dI, k=k, seed=HI + n)
+    _prefill_exact(w)
+
+
+def test_prefill_chunked_equals_whole():
+    w = W.scaled(W.PREFILL, B=1, n=1536, k=200, seed=77)
+    _prefill_exact(w, chunk=512)
+
+
+def test_prefill_scores_output_matches_oracle():
+    w = W.scaled(W.PREFILL, B=1, n=640, k=64, seed=9)
+    d = W.make_prefill_inputs(w, "cuda", with_attention=False)
+    ws = _ws()
+    idx, sc = dsa.indexer_topk_prefill(d["qI"], d["kI"], d["w"], w.k, return_scores=True, workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    q, k, wt = indexer_host_inputs(d)
+    full = O.indexer_scores(q, k, wt)
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    for i in range(w.n):
+        m = min(w.k, i + 1)
+        assert np.array_equal(sc[0, i, :m], full[0, i, idx[0, i, :m]])
+        assert np.all(np.isneginf(sc[0, i, m:]))
+
+
+def _prefill_tolerant(w, rows, chunk=None):
+    d = W.make_prefill_inputs(w, "cuda", with_attention=False)
+    ws = _ws()
+    kw = {}
+    if "q_scale" in d:
+        kw = dict(q_scale=d["q_scale"], k_scale=d["k_scale"])
+    if chunk is None:
+        idx = dsa.indexer_topk_prefill(d["qI"], d["kI"], d["w"], w.k, workspace=ws, **kw)
+    else:
+        idx = torch.empty((w.B, w.n, w.k), dtype=torch.int32, device="cuda")
+        for c0 in range(0, w.n, chunk):
+            c1 = min(w.n, c0 + chunk)
+            ckw = {}
+            if kw:
+                ckw = dict(q_scale=kw["q_scale"][:, c0:c1].contiguous(), k_scale=kw["k_scale"])
+            dsa.indexer_topk_prefill(d["qI"][:, c0:c1], d["kI"], d["w"][:, c0:c1], w.k, q_offset=c0,
+                                     idx_out=idx[:, c0:c1], workspace=ws, **ckw)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    idx = idx.cpu().numpy()
+    q, k, wt = indexer_host_inputs(d)
+    bad, overlaps = [], []
+    for b, i in rows:
+        s = O.indexer_scores_row(q[b, i], k[b, : i + 1], wt[b, i])
+        errs, st = checks.topk_tolerant_errors(idx[b, i], s, i, w.k)
+        bad += errs
+        overlaps.append(st["overlap"])
+    assert not bad, bad[:5]
+    return float(np.mean(overlaps))
+
+
+def test_prefill_fp8_small():
+    w = W.scaled(W.PREFILL_FP8, B=2, n=2304, k=256, seed=21)
+    ov = _prefill_tolerant(w, W.sample_rows(w, 96))
+    assert ov > 0.99
+
+
+def test_prefill_float_bf16_chunked():
+    w = W.scaled(W.LONG, n=4096, k=512, chunk=1024, seed=31)
+    ov = _prefill_tolerant(w, W.sample_rows(w, 96), chunk=1024)
+    assert ov > 0.99
+
+
+# --------------------------------------------------------------------------
+# eq. (3): sparse attention
+# --------------------------------------------------------------------------
+
+def _attn_check(q, latent, idx, out, lse, scale, dv, rows, atol=ATOL, rtol=RTOL):
+    qh, lh, ih = host_f64(q), host_f64(latent), idx.cpu().numpy()
+    oh, lseh = host_f64(out), lse.cpu().double().numpy()
+    bad = []
+    for b, i in rows:
+        ro, rl = O.sparse_attention_row(qh[b, i], lh[b], ih[b, i], scale, dv)
+        bad += checks.close_errors(oh[b, i], ro, atol, rtol, f"out[{b},{i}]")
+        bad += checks.close_errors(lseh[b, i], rl, 1e-3, 1e-3, f"lse[{b},{i}]")
+    assert not bad, bad[:5]
+
+
+def test_attention_tiny_full():
+    w = W.TINY
+    d = W.make_prefill_inputs(w, "cuda")
+    ws = _ws()
+    idx = dsa.indexer_topk_prefill(d["qI"], d["kI"], d["w"], w.k, workspace=ws)
+    out, lse = dsa.sparse_attn_prefill(d["q"], d["latent"], idx, w.Dv, scale=w.scale, return_lse=True, workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    _attn_check(d["q"], d["latent"], idx, out, lse, w.scale, w.Dv, [(0, i) for i in range(w.n)])
+
+
+def test_attention_mla_shapes_random_indices():
+    # 576/512 latent rows, 16 heads, random valid / -1 slots, ragged k
+    g = torch.Generator(device="cuda").manual_seed(3)
+    B, nq, kv, H, k = 2, 40, 3000, 16, 300
+    q = torch.randn((B, nq, H, 576), generator=g, device="cuda").bfloat16()
+    lat = torch.randn((B, kv, 576), generator=g, device="cuda").bfloat16()
+    idx = torch.randint(0, kv, (B, nq, k), generator=g, device="cuda", dtype=torch.int32)
+    idx[:, :, 250:] = -1
+    idx[0, 0, :] = -1                       # a row with nothing selected
+    idx[1, 3, 5:] = -1
+    ws = _ws()
+    out, lse = dsa.sparse_attn_prefill(q, lat, idx, 512, scale=1 / 24, return_lse=True, workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    assert torch.all(out[0, 0] == 0) and torch.all(torch.isneginf(lse[0, 0]))
+    _attn_check(q, lat, idx, out, lse, 1 / 24, 512, [(b, i) for b in range(B) for i in range(nq)])
+
+
+def test_attention_bad_index_is_reported_and_skipped():
+    B, nq, kv, H, k = 1, 4, 100, 16, 32
+    q = torch.randn((B, nq, H, 64), device="cuda").bfloat16()
+    lat = torch.randn((B, kv, 64), device="cuda").bfloat16()
+    idx = torch.randint(0, kv, (B, nq, k), device="cuda", dtype=torch.int32)
+    idx[0, 2, 7] = kv + 5
+    ws = _ws()
+    out, lse = dsa.sparse_attn_prefill(q, lat, idx, 64, scale=0.125, return_lse=True, workspace=ws)
+    st, detail = ws.status()
+    assert st == 6 and detail == 0xA77E
+    fixed = idx.clone()
+    fixed[0, 2, 7] = -1
+    _attn_check(q, lat, fixed, out, lse, 0.125, 64, [(0, i) for i in range(nq)])
+
+
+def test_worked_example_through_the_library():
+    """The page's three-token example (§1.1, eqs. (4)-(6)) embedded in padded
+    shapes: H_I 2 -> 4 and d_I 2 -> 32 with zero rows / weights (exact)."""
+    n, HI, dI = 3, 4, 32
+    qI = torch.zeros((1, n, HI, dI))
+    qI[0, 2, 0, 0] = 1.0
+    qI[0, 2, 1, 1] = 1.0
+    kI = torch.zeros((1, n, dI))
+    kI[0, :, :2] = torch.tensor([[2.0, -1.0], [1.0, 3.0], [-1.0, 4.0]])
+    w = torch.zeros((1, n, HI))
+    w[0, 2, :2] = torch.tensor([0.75, 0.25])
+    ws = _ws()
+    args = (qI.bfloat16().cuda(), kI.bfloat16().cuda(), w.cuda())
+    sc = dsa.indexer_scores(*args, workspace=ws)
+    assert sc[0, 2].tolist() == [1.5, 1.5, 1.0]
+    idx, val = dsa.indexer_topk_prefill(*args, 2, return_scores=True, workspace=ws)
+    assert sorted(idx[0, 2].tolist()) == [0, 1]
+    assert sorted(val[0, 2].tolist()) == [1.5, 1.5]
+    idx1 = dsa.indexer_topk_prefill(*args, 1, workspace=ws)
+    assert idx1[0, 2].tolist() == [0]
+    # attention half: logits 0.2 / 1.2 on values (2,0) / (0,3), through a
+    # constructed latent row c_s = (v_s, 0.., a_s) and q = (0.., 1), scale 1
+    lat = torch.zeros((1, n, 64))
+    lat[0, 0, :2] = torch.tensor([2.0, 0.0])
+    lat[0, 1, :2] = torch.tensor([0.0, 3.0])
+    lat[0, :, 63] = torch.tensor([0.2, 1.2, 2.0])
+    q = torch.zeros((1, n, 1, 64))
+    q[0, :, 0, 63] = 1.0
+    out = dsa.sparse_attn_prefill(q.bfloat16().cuda(), lat.bfloat16().cuda(), idx, 64, scale=1.0, workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    o = out[0, 2, 0, :2].float().cpu().numpy()
+    assert np.allclose(o, [0.538, 2.193], atol=1e-2)          # bf16 logits 0.2002 / 1.2031
+
+
+# --------------------------------------------------------------------------
+# decode
+# --------------------------------------------------------------------------
+
+def _decode_case(w, lengths, fp8=False):
+    d = W.make_decode_inputs(w, "cuda", lengths=lengths)
+    total, maxlen = int(lengths.sum()), int(lengths.max())
+    ws = _ws()
+    idx = dsa.indexer_topk_decode(d["qI"], d["w"], d["kI_cache"], d["cu_seqlens"], w.k, total, maxlen, workspace=ws)
+    out, lse = dsa.sparse_attn_decode(d["q"], d["latent_cache"], d["cu_seqlens"], idx, w.Dv, total, scale=w.scale,
+                                      return_lse=True, workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    cu = d["cu_seqlens"].cpu().numpy()
+    qh, kh, wh = host_f64(d["qI"]), host_f64(d["kI_cache"]), host_f64(d["w"])
+    idx_h = idx.cpu().numpy()
+    bad = []
+    for b in range(len(lengths)):
+        s = O.indexer_scores_row(qh[b], kh[cu[b]:cu[b + 1]], wh[b])
+        errs, _ = checks.topk_tolerant_errors(idx_h[b], s, int(lengths[b]) - 1, w.k)
+        bad += errs
+    assert not bad, bad[:5]
+    ro, rl = O.decode_sparse_attention(host_f64(d["q"]), host_f64(d["latent_cache"]), cu, idx_h, w.scale, w.Dv)
+    bad = checks.close_errors(host_f64(out), ro, ATOL, RTOL, "decode out")
+    bad += checks.close_errors(lse.cpu().double().numpy(), rl, 1e-3, 1e-3, "decode lse")
+    assert not bad, bad
+
+
+def test_decode_small_ragged():
+    w = W.scaled(W.DECODE, B=5, k=300)
+    _decode_case(w, torch.tensor([1, 129, 300, 1000, 4097]))
+
+
+@pytest.mark.slow
+def test_decode_full_workload():
+    _decode_case(W.DECODE, W.decode_lengths(W.DECODE))
+
+
+# --------------------------------------------------------------------------
+# full-size workloads, sampled rows
+# --------------------------------------------------------------------------
+
+@pytest.mark.slow
+def test_prefill_full_integer_workload_sampled():
+    w = W.PREFILL
+    _prefill_exact(w, rows=W.sample_rows(w, 256))
+
+
+@pytest.mark.slow
+def test_prefill_full_fp8_workload_sampled():
+    w = W.PREFILL_FP8
+    ov = _prefill_tolerant(w, W.sample_rows(w, 256))
+    assert ov > 0.98
+
+
+@pytest.mark.slow
+def test_long_prefill_chunked_sampled():
+    w = W.LONG
+    ov = _prefill_tolerant(w, W.sample_rows(w, 64), chunk=w.chunk)
+    assert ov > 0.98
+
+
+@pytest.mark.slow
+def test_attention_full_prefill_sampled():
+    w = W.PREFILL
+    d = W.make_prefill_inputs(w, "cuda")
+    ws = _ws()
+    idx = dsa.indexer_topk_prefill(d["qI"], d["kI"], d["w"], w.k, workspace=ws)
+    out, lse = dsa.sparse_attn_prefill(d["q"], d["latent"], idx, w.Dv, scale=w.scale, return_lse=True, workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    _attn_check(d["q"], d["latent"], idx, out, lse, w.scale, w.Dv, W.sample_rows(w, 128))
