@@ -111,7 +111,8 @@ dsa_status dsa_indexer_topk_prefill(int B, int nq, int q_offset, int kv_len, int
  *   out    [B, nq, H, Dv]   bf16      lse [B, nq, H] fp32 or NULL
  * A row with no valid slot gives out = 0, lse = -inf.  An index outside
  * [-1, kv_len) is skipped and recorded as DSA_ERR_DEVICE_CHECK.
- * Supported: Dqk a multiple of 16, <= 1024; Dv in {64,128,256,512}, Dv <= Dqk.
+ * Supported: Dqk a multiple of 16, <= 576; Dv a multiple of 64, <= min(512, Dqk);
+ * k <= 2048.
  * ---------------------------------------------------------------------- */
 size_t dsa_sparse_attn_workspace(void);
 dsa_status dsa_sparse_attn_prefill(int B, int nq, int kv_len, int H, int Dqk, int Dv, int k, float scale,

@@ -225,13 +225,32 @@ dsa_status dsa_indexer_topk_prefill(int B, int nq, int q_offset, int kv_len, int
 static dsa_status check_attn(int H, int Dqk, int Dv, int k, const void* q, const void* lat, const int32_t* idx,
                              const void* out, const float* lse) {
   DSA_CHECK(H >= 1 && k >= 1, DSA_ERR_INVALID_ARG, "need H >= 1 and k >= 1");
-  DSA_CHECK(Dqk % 16 == 0 && Dqk >= 16 && Dqk <= 1024, DSA_ERR_UNSUPPORTED,
-            "Dqk=%d: must be a multiple of 16 in [16, 1024]", Dqk);
-  DSA_CHECK((Dv == 64 || Dv == 128 || Dv == 256 || Dv == 512) && Dv <= Dqk, DSA_ERR_UNSUPPORTED,
-            "Dv=%d: supported 64, 128, 256, 512 and Dv <= Dqk", Dv);
+  DSA_CHECK(k <= 2048, DSA_ERR_UNSUPPORTED, "k=%d: sparse attention supports k <= 2048", k);
+  DSA_CHECK(Dqk % 16 == 0 && Dqk >= 16 && Dqk <= 576, DSA_ERR_UNSUPPORTED,
+            "Dqk=%d: must be a multiple of 16 in [16, 576]", Dqk);
+  DSA_CHECK(Dv % 64 == 0 && Dv >= 64 && Dv <= 512 && Dv <= Dqk, DSA_ERR_UNSUPPORTED,
+            "Dv=%d: must be a multiple of 64 in [64, 512] and <= Dqk", Dv);
   DSA_CHECK(q && lat && idx && out, DSA_ERR_INVALID_ARG, "null tensor pointer");
   DSA_CHECK(aligned(q, 16) && aligned(lat, 16) && aligned(idx, 4) && aligned(out, 4) && aligned(lse, 4),
             DSA_ERR_INVALID_ARG, "q and latent must be 16-byte aligned");
+  return DSA_OK;
+}
+
+static dsa_status run_attn(dsa::AttnArgs& a, const void* q, const void* latent, int64_t latent_rows,
+                           cudaStream_t s) {
+  a.nh = 16;
+  a.cb = (a.Dqk + 63) / 64;
+  a.ksteps = a.Dqk / 16;
+  a.dv_tiles = a.Dv / 64;
+  a.timeout_ns = g_timeout_ns;
+  DSA_CHECK((int64_t)a.rows * a.H < INT32_MAX && latent_rows < INT32_MAX, DSA_ERR_UNSUPPORTED,
+            "tensor rows exceed 2^31");
+  (void)q;
+  (void)latent;
+  const int64_t items = (int64_t)a.rows * ((a.H + a.nh - 1) / a.nh);
+  const int grid = (int)std::min<int64_t>(sm_count(), items);
+  cudaError_t e = dsa::launch_sparse_attn(a, grid, s);
+  if (e != cudaSuccess) return cuda_fail(e, "sparse_attn launch");
   return DSA_OK;
 }
 
@@ -260,9 +279,7 @@ dsa_status dsa_sparse_attn_prefill(int B, int nq, int kv_len, int H, int Dqk, in
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
   a.status = status_of(workspace);
-  cudaError_t e = dsa::launch_sparse_attn(a, (cudaStream_t)stream);
-  if (e != cudaSuccess) return cuda_fail(e, "sparse_attn launch");
-  return DSA_OK;
+  return run_attn(a, q, latent, (int64_t)B * kv_len, (cudaStream_t)stream);
 }
 
 dsa_status dsa_sparse_attn_decode(int B, int H, int Dqk, int Dv, int k, float scale, const void* q,
@@ -270,7 +287,7 @@ dsa_status dsa_sparse_attn_decode(int B, int H, int Dqk, int Dv, int k, float sc
                                   const int32_t* idx, void* out, float* lse, void* workspace,
                                   size_t workspace_bytes, void* stream) {
   if (dsa_status st = check_attn(H, Dqk, Dv, k, q, latent_cache, idx, out, lse)) return st;
-  DSA_CHECK(B >= 0 && cu_seqlens && total_len >= 0, DSA_ERR_INVALID_ARG, "need B >= 0, cu_seqlens, total_len >= 0");
+  DSA_CHECK(B >= 0 && cu_seqlens && total_len >= 1, DSA_ERR_INVALID_ARG, "need B >= 0, cu_seqlens, total_len >= 1");
   DSA_CHECK(std::isfinite(scale), DSA_ERR_INVALID_ARG, "scale must be finite");
   if (dsa_status st = check_ws(workspace, workspace_bytes, kHeader)) return st;
   if (B == 0) return DSA_OK;
@@ -290,9 +307,7 @@ dsa_status dsa_sparse_attn_decode(int B, int H, int Dqk, int Dv, int k, float sc
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
   a.status = status_of(workspace);
-  cudaError_t e = dsa::launch_sparse_attn(a, (cudaStream_t)stream);
-  if (e != cudaSuccess) return cuda_fail(e, "sparse_attn (decode) launch");
-  return DSA_OK;
+  return run_attn(a, q, latent_cache, total_len, (cudaStream_t)stream);
 }
 
 // ---------------------------------------------------------------- decode indexer

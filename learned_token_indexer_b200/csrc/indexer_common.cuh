@@ -69,4 +69,58 @@ __device__ __forceinline__ float relu_weighted_head_sum(const uint32_t (&acc)[HI
   return s;
 }
 
+// Eq. (1) for TOK consecutive tokens of one accumulator (columns
+// [j*HI, (j+1)*HI) hold token j's heads) and this thread's key.  TMEM is read
+// in units of up to 32 columns, loading unit u+1 while unit u is reduced; each
+// token keeps 4 independent partial sums so the FMA chain does not serialise.
+// After the last load the accumulator is handed back (`acc_empty`, one arrive
+// per warp) before the last unit is reduced.
+template <int HI, int TOK>
+__device__ __forceinline__ void group_head_sums(uint32_t taddr, const float* w_smem, float (&score)[TOK],
+                                                uint64_t* acc_empty, uint32_t lane) {
+  constexpr int UW = HI < 32 ? HI : 32;      // columns per unit
+  constexpr int UPT = HI / UW;               // units per token
+  constexpr int NU = TOK * UPT;
+  float2 part[TOK][2];
+#pragma unroll
+  for (int j = 0; j < TOK; ++j) part[j][0] = part[j][1] = make_float2(0.0f, 0.0f);
+  uint32_t buf[2][UW];
+  auto load = [&](int u, uint32_t (&r)[UW]) {
+    const uint32_t col = (uint32_t)((u / UPT) * HI + (u % UPT) * UW);
+    if constexpr (UW == 4) tmem_ld_32x32b_x4(taddr + col, r);
+    else if constexpr (UW == 8) tmem_ld_32x32b_x8(taddr + col, r);
+    else if constexpr (UW == 16) tmem_ld_32x32b_x16(taddr + col, r);
+    else tmem_ld_32x32b_x32(taddr + col, r);
+  };
+  load(0, buf[0]);
+  tmem_wait_ld(buf[0]);
+#pragma unroll
+  for (int u = 0; u < NU; ++u) {
+    if (u + 1 < NU) load(u + 1, buf[(u + 1) & 1]);
+    const int j = u / UPT;
+    const float2* w = reinterpret_cast<const float2*>(w_smem + j * HI + (u % UPT) * UW);
+#pragma unroll
+    for (int h = 0; h < UW; h += 2) {
+      const float2 x = make_float2(fmaxf(__uint_as_float(buf[u & 1][h]), 0.0f),
+                                   fmaxf(__uint_as_float(buf[u & 1][h + 1]), 0.0f));
+      part[j][(h >> 1) & 1] = ffma2(w[h >> 1], x, part[j][(h >> 1) & 1]);
+    }
+    if (u + 1 < NU) {
+      tmem_wait_ld(buf[(u + 1) & 1]);
+      if (u + 2 == NU) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+      }
+    }
+  }
+  if (NU == 1) {
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(acc_empty);
+  }
+#pragma unroll
+  for (int j = 0; j < TOK; ++j) score[j] = (part[j][0].x + part[j][1].x) + (part[j][0].y + part[j][1].y);
+}
+
 }  // namespace dsa

@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           tc_fence_after();
           uint32_t r[HI];
           tmem_load_heads<HI>(tmem_base + (lane_grp << 16) + acc * N, r);
-          tmem_wait_ld();
+          tmem_wait_ld(r);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[acc]);

@@ -6,11 +6,12 @@
 //
 // Work unit: a block of 8 consecutive query tokens of one sequence against
 // all keys 0..t of its last token.  Persistent grid, heavy blocks first, snake
-// order over CTAs.  Per CTA (10 warps):
+// order over CTAs.  Per CTA (18 warps):
 //   warp 0      TMA producer: Q of the block (both groups, once), K tiles;
 //   warp 1      tcgen05 MMA issuer, TMEM owner: for each 128-key tile and
 //               each group g of 4 tokens, D_g[128 keys x 4*HI] (+)= K Q_g^T;
-//   warps 2..5  epilogue group 0 (tokens 0..3), warps 6..9 group 1 (4..7):
+//   warps 2..17 epilogue, 4 warpgroups; warpgroup j takes token j of group 0
+//               and token 4+j of group 1 (both accumulators, in MMA order):
 //               TMEM -> ReLU * w -> head sum = I[t, s]; causal mask; then
 //               the streaming filter below; after the block's last tile the
 //               exact select (select.cuh) writes idx (and scores).
@@ -30,7 +31,7 @@ namespace {
 
 constexpr int kQB = 8;          // tokens per block
 constexpr int kTA = 4;          // tokens per accumulator group
-constexpr int kPrefillThreads = 320;
+constexpr int kPrefillThreads = 576;   // producer, MMA, 4 epilogue warpgroups
 constexpr int kHistBins = 512;  // streaming histogram bins (499 used)
 constexpr uint32_t kLastBin = 498;
 
@@ -106,9 +107,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint32_t* sCount = sHist + kQB * kHistBins;                             // [8]
   uint32_t* sFloor = sCount + kQB;                                        // [8]
   uint32_t* sBelow = sFloor + kQB;                                        // [8]
-  SelectShared<128>* sSel = reinterpret_cast<SelectShared<128>*>(sBelow + kQB);  // [2]
+  SelectShared<128>* sSel = reinterpret_cast<SelectShared<128>*>(sBelow + kQB);  // [4]
   uint64_t* bars = reinterpret_cast<uint64_t*>(
-      (reinterpret_cast<uintptr_t>(sSel + 2) + 7) & ~uintptr_t(7));
+      (reinterpret_cast<uintptr_t>(sSel + 4) + 7) & ~uintptr_t(7));
   uint64_t* k_full = bars;
   uint64_t* k_empty = bars + STAGES;
   uint64_t* q_full = bars + 2 * STAGES;
@@ -129,7 +130,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     mbar_init(q_empty, 1);
     for (int g = 0; g < 2; ++g) {
       mbar_init(&acc_full[g], 1);
-      mbar_init(&acc_empty[g], 4);
+      mbar_init(&acc_empty[g], 16);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0u;
@@ -237,115 +238,124 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
-    // Every thread of a group runs the same sequence of named barriers; a
+    // Four warpgroups; warpgroup j owns block token j of accumulator group 0
+    // and token 4+j of group 1 (columns [j*HI, (j+1)*HI) of each group).
+    // Every thread of a warpgroup runs the same sequence of named barriers; a
     // wait that fails only turns the remaining work into no-ops (no early
     // exit, so no barrier is ever left short of threads).
-    const uint32_t g = (warp - 2) >> 2;                  // accumulator group 0/1
-    const uint32_t tid = (warp - 2 - 4 * g) * 32 + lane; // 0..127 inside the group
-    const uint32_t bar_id = 2 + g;
+    const uint32_t wg = (warp - 2) >> 2;                  // 0..3
+    const uint32_t tid = (warp - 2 - 4 * wg) * 32 + lane; // 0..127 inside the warpgroup
+    const uint32_t bar_id = 2 + wg;
     const uint32_t lane_grp = (warp & 3u) * 32u;
     const uint32_t key_in_tile = lane_grp + lane;
-    SelectShared<128>& sel = sSel[g];
-    uint32_t aphase = 0;
+    SelectShared<128>& sel = sSel[wg];
+    uint32_t aphase[2] = {0u, 0u};
     bool ok = true;
     Block blk;
     for (int r = 0; block_of(a, r, blk); ++r) {
       named_bar_sync(bar_id, 128);
-      // per-block state of this group's 4 tokens
-      int tok_t[kTA];
-      bool tok_valid[kTA];
+      // per-block state of this warpgroup's 2 tokens (slot st = 4*g + wg)
+      int tok_t[2];
+      bool tok_valid[2];
 #pragma unroll
-      for (int j = 0; j < kTA; ++j) {
-        const int li = blk.t0 + kTA * (int)g + j;
-        tok_valid[j] = li < a.nq;
-        tok_t[j] = a.q_offset + li;
+      for (int g = 0; g < 2; ++g) {
+        const int li = blk.t0 + kTA * g + (int)wg;
+        tok_valid[g] = li < a.nq;
+        tok_t[g] = a.q_offset + li;
       }
-      for (int i = (int)tid; i < kTA * kHistBins; i += 128) sHist[(kTA * g) * kHistBins + i] = 0u;
-      if (tid < (uint32_t)kTA) {
-        sCount[kTA * g + tid] = 0u;
-        sFloor[kTA * g + tid] = 0u;
-        sBelow[kTA * g + tid] = 0u;
+      for (int i = (int)tid; i < 2 * kHistBins; i += 128) {
+        const int g = i / kHistBins;
+        sHist[(kTA * g + wg) * kHistBins + (i - g * kHistBins)] = 0u;
       }
-      for (int i = (int)tid; i < kTA * HI; i += 128) {
-        const int j = i / HI, h = i - j * HI;
-        const int li = blk.t0 + kTA * (int)g + j;
+      if (tid < 2u) {
+        sCount[kTA * tid + wg] = 0u;
+        sFloor[kTA * tid + wg] = 0u;
+        sBelow[kTA * tid + wg] = 0u;
+      }
+      for (int i = (int)tid; i < 2 * HI; i += 128) {
+        const int g = i / HI, h = i - g * HI;
+        const int li = blk.t0 + kTA * g + (int)wg;
         float wv = 0.0f;
         if (li < a.nq) {
           const int64_t row = (int64_t)blk.b * a.nq + li;
           wv = a.w[row * HI + h];
           if (FP8) wv *= a.q_scale[row];
         }
-        sW[(kTA * g + j) * HI + h] = wv;
+        sW[(kTA * g + wg) * HI + h] = wv;
       }
       named_bar_sync(bar_id, 128);
-      const int nt = blk.nt[g];
-      uint2* cand_base = a.cand + ((int64_t)blockIdx.x * kQB + kTA * g) * a.cand_cap;
-      for (int t = 0; t < nt; ++t) {
-        bool got = ok && mbar_wait(&acc_full[g], aphase, ctl, 0x1301);
-        ok = __all_sync(0xffffffffu, got);
-        aphase ^= 1u;
-        const int s = t * kTileKeys + (int)key_in_tile;
-        float score[kTA];
-        if (ok) {
-          tc_fence_after();
-          float ks = 1.0f;
-          if (FP8) ks = (s < a.kv_len) ? a.k_scale[(int64_t)blk.b * a.kv_len + s] : 0.0f;
+      const int nt_max = max(blk.nt[0], blk.nt[1]);
+      uint2* cand_tok[2];
 #pragma unroll
-          for (int j = 0; j < kTA; ++j) {
-            uint32_t rr[HI];
-            tmem_load_heads<HI>(tmem_base + (lane_grp << 16) + g * N + j * HI, rr);
-            tmem_wait_ld();
-            score[j] = relu_weighted_head_sum<HI>(rr, sW + (kTA * g + j) * HI);
-            if (FP8) score[j] *= ks;
+      for (int g = 0; g < 2; ++g)
+        cand_tok[g] = a.cand + ((int64_t)blockIdx.x * kQB + kTA * g + wg) * a.cand_cap;
+      for (int t = 0; t < nt_max; ++t) {
+        const int s = t * kTileKeys + (int)key_in_tile;
+        float ks = 1.0f;
+        if (FP8 && ok) ks = (s < a.kv_len) ? a.k_scale[(int64_t)blk.b * a.kv_len + s] : 0.0f;
+        float score[2] = {0.0f, 0.0f};
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          if (t >= blk.nt[g]) continue;
+          const bool got = ok && mbar_wait(&acc_full[g], aphase[g], ctl, 0x1301);
+          ok = __all_sync(0xffffffffu, got);
+          aphase[g] ^= 1u;
+          if (ok) {
+            tc_fence_after();
+            float sc[1];
+            group_head_sums<HI, 1>(tmem_base + (lane_grp << 16) + g * N + wg * HI, sW + (kTA * g + wg) * HI, sc,
+                                   &acc_empty[g], lane);
+            score[g] = FP8 ? sc[0] * ks : sc[0];
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[g]);
         }
         named_bar_sync(bar_id, 128);     // previous tile's floor update is visible
         if (ok) {
 #pragma unroll
-          for (int j = 0; j < kTA; ++j) {
-            const uint32_t key = float_to_key(score[j]);
+          for (int g = 0; g < 2; ++g) {
+            if (t >= blk.nt[g]) continue;
+            const int st = kTA * g + (int)wg;
+            const uint32_t key = float_to_key(score[g]);
             const uint32_t bin = score_bin(key);
-            const bool acc = tok_valid[j] && s <= tok_t[j] && bin >= sFloor[kTA * g + j];
+            const bool acc = tok_valid[g] && s <= tok_t[g] && bin >= sFloor[st];
             const uint32_t mask = __ballot_sync(0xffffffffu, acc);
             if (mask) {
               uint32_t slot0 = 0;
-              if (lane == 0) slot0 = atomicAdd(&sCount[kTA * g + j], (uint32_t)__popc(mask));
+              if (lane == 0) slot0 = atomicAdd(&sCount[st], (uint32_t)__popc(mask));
               slot0 = __shfl_sync(0xffffffffu, slot0, 0);
               if (acc) {
                 const uint32_t slot = slot0 + __popc(mask & ((1u << lane) - 1u));
-                cand_base[(int64_t)j * a.cand_cap + slot] = make_uint2(key, (uint32_t)s);
-                atomicAdd(&sHist[(kTA * g + j) * kHistBins + bin], 1u);
+                cand_tok[g][slot] = make_uint2(key, (uint32_t)s);
+                atomicAdd(&sHist[st * kHistBins + bin], 1u);
               }
             }
           }
         }
         named_bar_sync(bar_id, 128);     // this tile's appends are complete
-        if (ok && tid < (uint32_t)kTA) {
-          const uint32_t* h = sHist + (kTA * g + tid) * kHistBins;
-          const uint32_t c = sCount[kTA * g + tid];
-          uint32_t fl = sFloor[kTA * g + tid], bl = sBelow[kTA * g + tid];
+        if (ok && tid < 2u && t < blk.nt[tid]) {
+          const int st = kTA * (int)tid + (int)wg;
+          const uint32_t* h = sHist + st * kHistBins;
+          const uint32_t c = sCount[st];
+          uint32_t fl = sFloor[st], bl = sBelow[st];
           while (fl < kLastBin && c - bl - h[fl] >= (uint32_t)a.k) {
             bl += h[fl];
             ++fl;
           }
-          sFloor[kTA * g + tid] = fl;
-          sBelow[kTA * g + tid] = bl;
+          sFloor[st] = fl;
+          sBelow[st] = bl;
         }
       }
       named_bar_sync(bar_id, 128);
       if (tid == 0) sel.aborted = *abort_flag;
       named_bar_sync(bar_id, 128);
-      if (sel.aborted) continue;   // group-uniform: nothing below is valid
+      if (sel.aborted) continue;   // warpgroup-uniform: nothing below is valid
       // ---- exact select of each token's top min(k, t+1)
-      for (int j = 0; j < kTA; ++j) {
-        if (!tok_valid[j] || nt == 0) continue;
-        const int kk = min(a.k, tok_t[j] + 1);
-        const int m = (int)sCount[kTA * g + j];
-        uint32_t* hist = sHist + (kTA * g + j) * kHistBins;
-        const uint2* buf = cand_base + (int64_t)j * a.cand_cap;
+      for (int g = 0; g < 2; ++g) {
+        if (!tok_valid[g] || blk.nt[g] == 0) continue;
+        const int st = kTA * g + (int)wg;
+        const int kk = min(a.k, tok_t[g] + 1);
+        const int m = (int)sCount[st];
+        uint32_t* hist = sHist + st * kHistBins;
+        const uint2* buf = cand_tok[g];
         auto get = [buf](int i, uint32_t& key, uint32_t& pos) {
           const uint2 e = buf[i];
           key = e.x;
@@ -361,9 +371,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         res.key_all_in = 1;
         res.pos_hi = 0;
         if (need != cnt)
-          res = group_refine<128, kHistBins>(get, m, res.lo, res.hi, need, (uint32_t)tok_t[j], hist, sel, tid,
+          res = group_refine<128, kHistBins>(get, m, res.lo, res.hi, need, (uint32_t)tok_t[g], hist, sel, tid,
                                              bar_id);
-        const int64_t row = (int64_t)blk.b * a.nq + blk.t0 + kTA * g + j;
+        const int64_t row = (int64_t)blk.b * a.nq + blk.t0 + st;
         group_emit<128>(get, m, res, kk, a.k, a.idx_out + row * a.k,
                         a.score_out ? a.score_out + row * a.k : nullptr, sel, tid, bar_id, a.status);
       }
@@ -386,7 +396,7 @@ struct PrefillConfig {
   static constexpr int kQBytes = 2 * N * KB * kSwizzleBytes;
   static constexpr int kKBytes = kTileKeys * KB * kSwizzleBytes;
   static constexpr int kFixed = 1024 /*align*/ + kQBytes + kQB * HI * 4 + kQB * kHistBins * 4 + 3 * kQB * 4 +
-                                2 * (int)sizeof(SelectShared<128>) + 8 + 16 * 8 + 16;
+                                4 * (int)sizeof(SelectShared<128>) + 8 + 16 * 8 + 16;
   static constexpr int kBudget = 227 * 1024;
   static constexpr int kStagesFit = (kBudget - kFixed) / kKBytes;
   static constexpr int STAGES = kStagesFit > 6 ? 6 : kStagesFit;

@@ -59,6 +59,11 @@ struct TopkRowsArgs {
 struct AttnArgs {
   int rows;                    // query rows (prefill B*nq, decode B)
   int H, Dqk, Dv, k;
+  int nh;                      // heads per CTA (MMA N)
+  int cb;                      // 64-column blocks per latent row
+  int ksteps;                  // 16-column K steps of the logits MMA (Dqk / 16)
+  int dv_tiles;                // 64-wide value tiles (Dv / 64)
+  uint64_t timeout_ns;
   float scale_log2;            // softmax scale * log2(e)
   float scale;
   const uint16_t* q;           // [rows, H, Dqk] bf16
@@ -81,7 +86,7 @@ cudaError_t launch_topk_rows(const TopkRowsArgs& a, cudaStream_t stream);
 cudaError_t launch_fill_trivial_rows(int B, int nq, int q_offset, int rows_per_seq, int k, int32_t* idx,
                                      cudaStream_t stream);
 cudaError_t launch_fill_f32(float* p, int64_t n, float v, cudaStream_t stream);
-cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t stream);
+cudaError_t launch_sparse_attn(const AttnArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_wait_selftest(DeviceStatus* status, uint64_t timeout_ns, cudaStream_t stream);
 
 }  // namespace dsa

@@ -22,6 +22,10 @@
 
 namespace dsa {
 
+// Entries read per thread per pass before they are processed (independent
+// loads in flight).
+constexpr int kBatch = 8;
+
 struct SelectResult {
   uint32_t lo, hi;        // key interval of the cut-off
   uint32_t key_all_in;    // 1: every entry with key >= lo is selected
@@ -93,10 +97,17 @@ __device__ SelectResult group_refine(Get get, int m, uint32_t lo, uint32_t hi, u
     const int nb = (int)((hi >> s) - base) + 1;
     for (int i = (int)tid; i < nb; i += NT) hist[i] = 0u;
     named_bar_sync(bar_id, NT);
-    for (int i = (int)tid; i < m; i += NT) {
-      uint32_t key, pos;
-      get(i, key, pos);
-      if (key >= lo && key <= hi) atomicAdd(&hist[(key >> s) - base], 1u);
+    for (int i0 = (int)tid; i0 < m; i0 += NT * kBatch) {
+      uint32_t key[kBatch], pos[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        key[u] = 0u;
+        pos[u] = 0u;
+        if (i0 + u * NT < m) get(i0 + u * NT, key[u], pos[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        if (i0 + u * NT < m && key[u] >= lo && key[u] <= hi) atomicAdd(&hist[(key[u] >> s) - base], 1u);
     }
     named_bar_sync(bar_id, NT);
     group_find<NT>(hist, nb, need, true, sh, tid, bar_id);
@@ -126,10 +137,18 @@ __device__ SelectResult group_refine(Get get, int m, uint32_t lo, uint32_t hi, u
     const int nb = (int)((phi >> s) - base) + 1;
     for (int i = (int)tid; i < nb; i += NT) hist[i] = 0u;
     named_bar_sync(bar_id, NT);
-    for (int i = (int)tid; i < m; i += NT) {
-      uint32_t key, pos;
-      get(i, key, pos);
-      if (key == lo && pos >= plo && pos <= phi) atomicAdd(&hist[(pos >> s) - base], 1u);
+    for (int i0 = (int)tid; i0 < m; i0 += NT * kBatch) {
+      uint32_t key[kBatch], pos[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        key[u] = 0u;
+        pos[u] = 0u;
+        if (i0 + u * NT < m) get(i0 + u * NT, key[u], pos[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        if (i0 + u * NT < m && key[u] == lo && pos[u] >= plo && pos[u] <= phi)
+          atomicAdd(&hist[(pos[u] >> s) - base], 1u);
     }
     named_bar_sync(bar_id, NT);
     group_find<NT>(hist, nb, need, false, sh, tid, bar_id);
@@ -163,23 +182,29 @@ __device__ void group_emit(Get get, int m, const SelectResult& r, int kk, int k,
   if (tid == 0) sh.out_count = 0;
   named_bar_sync(bar_id, NT);
   const uint32_t lane = tid & 31u;
-  for (int i0 = 0; i0 < m; i0 += NT) {
-    const int i = i0 + (int)tid;
-    uint32_t key = 0, pos = 0;
-    bool sel = false;
-    if (i < m) {
-      get(i, key, pos);
-      sel = selected(r, key, pos);
+  for (int j0 = 0; j0 < m; j0 += NT * kBatch) {
+    uint32_t key[kBatch], pos[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      key[u] = 0u;
+      pos[u] = 0u;
+      const int i = j0 + u * NT + (int)tid;
+      if (i < m) get(i, key[u], pos[u]);
     }
-    const uint32_t mask = __ballot_sync(0xffffffffu, sel);
-    uint32_t base = 0;
-    if (lane == 0 && mask) base = atomicAdd(&sh.out_count, (uint32_t)__popc(mask));
-    base = __shfl_sync(0xffffffffu, base, 0);
-    if (sel) {
-      const uint32_t slot = base + __popc(mask & ((1u << lane) - 1u));
-      if (slot < (uint32_t)kk) {
-        idx_row[slot] = (int32_t)pos;
-        if (score_row) score_row[slot] = key_to_float(key);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = j0 + u * NT + (int)tid;
+      const bool sel = i < m && selected(r, key[u], pos[u]);
+      const uint32_t mask = __ballot_sync(0xffffffffu, sel);
+      uint32_t base = 0;
+      if (lane == 0 && mask) base = atomicAdd(&sh.out_count, (uint32_t)__popc(mask));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (sel) {
+        const uint32_t slot = base + __popc(mask & ((1u << lane) - 1u));
+        if (slot < (uint32_t)kk) {
+          idx_row[slot] = (int32_t)pos[u];
+          if (score_row) score_row[slot] = key_to_float(key[u]);
+        }
       }
     }
   }
