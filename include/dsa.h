@@ -138,6 +138,34 @@ dsa_status dsa_indexer_topk_decode(int B, int HI, int dI, int k, int dtype, cons
                                    const int64_t* cu_seqlens, int64_t total_len, int max_len, int32_t* idx_out,
                                    float* score_out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* dsa_indexer_topk_decode_noalloc: the same decode-step selection as
+ * dsa_indexer_topk_decode (same arguments, same results), for callers that
+ * cannot allocate device memory and so cannot pass a workspace: for example
+ * a component inside a host runtime that owns every device allocation and
+ * hands it only its input and output buffers, or code called where no
+ * allocator is reachable.  The paper has no counterpart; this is a calling
+ * convenience of this library.
+ *   Scratch: a buffer built into the library (256 B status word + one fp32
+ *   score per cached key), a fixed 16 MiB + 256 B that every GPU which loads
+ *   the library holds until the process exits.  Nothing is allocated.
+ *   Limit: total_len <= 4,194,304 (2^22) cached keys over all B sequences;
+ *   larger steps return DSA_ERR_UNSUPPORTED with a message naming the limit.
+ *   Set-up: the first call made with a given device current looks up that
+ *   device's copy of the buffer (a host-side step); make that first call
+ *   before any stream capture.
+ *   Sharing: every call uses the same buffer, which keeps the last call's
+ *   contents; the status word is cleared at the start of each call (the
+ *   scores are fully rewritten).  Calls whose work overlaps on the GPU (two
+ *   streams, two threads) race on the buffer: order them on one stream.
+ *   status_out: NULL, or 2 device uint32 that receive this call's device
+ *   status word (code, detail; code 0 = success, else a dsa_status value),
+ *   copied on the stream after the kernels. */
+dsa_status dsa_indexer_topk_decode_noalloc(int B, int HI, int dI, int k, int dtype, const void* qI,
+                                           const float* q_scale, const float* w, const void* kI_cache,
+                                           const float* k_scale, const int64_t* cu_seqlens, int64_t total_len,
+                                           int max_len, int32_t* idx_out, float* score_out, uint32_t* status_out,
+                                           void* stream);
+
 /*   q [B, H, Dqk] bf16, latent_cache [total_len, Dqk] bf16, idx [B, k] local
  *   positions or -1, out [B, H, Dv] bf16, lse [B, H] fp32 or NULL. */
 dsa_status dsa_sparse_attn_decode(int B, int H, int Dqk, int Dv, int k, float scale, const void* q,

@@ -192,6 +192,22 @@ def indexer_topk_decode(qI, w, kI_cache, cu_seqlens, k: int, total_len: int, max
     return (idx_out, score_out) if score_out is not None else idx_out
 
 
+def indexer_topk_decode_noalloc(qI, w, kI_cache, cu_seqlens, k: int, total_len: int, max_len: int, idx_out,
+                                score_out=None, status_out=None, q_scale=None, k_scale=None):
+    """indexer_topk_decode for callers that cannot allocate device memory:
+    the library's built-in scratch (at most 2^22 cached keys per call) takes
+    the place of the workspace, and every output buffer is the caller's.
+    status_out, if given, is a device uint32 [2] that receives the call's
+    device status word. Calls that overlap on the GPU share that scratch and
+    race; order them on one stream."""
+    B, HI, dI = qI.shape
+    _check(lib().dsa_indexer_topk_decode_noalloc(B, HI, dI, k, _dtype_code(qI), _ptr(qI), _ptr(q_scale), _ptr(w),
+                                                 _ptr(kI_cache), _ptr(k_scale), _ptr(cu_seqlens), int(total_len),
+                                                 int(max_len), _ptr(idx_out), _ptr(score_out), _ptr(status_out),
+                                                 _stream(qI.device)))
+    return (idx_out, score_out) if score_out is not None else idx_out
+
+
 def sparse_attn_decode(q, latent_cache, cu_seqlens, idx, dv: int, total_len: int, scale: Optional[float] = None,
                        out=None, lse=None, return_lse: bool = False, workspace: Optional[Workspace] = None):
     """Eq. (3) for a decode step: q [B, H, Dqk], latent_cache [total_len, Dqk],

@@ -24,6 +24,7 @@ SIGNATURES = {
     "dsa_sparse_attn_prefill": (_i, [_i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "dsa_indexer_topk_decode_workspace": (_sz, [_i, _i, _i, _i, _i, _i64, _i]),
     "dsa_indexer_topk_decode": (_i, [_i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _i64, _i, _p, _p, _p, _sz, _p]),
+    "dsa_indexer_topk_decode_noalloc": (_i, [_i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _i64, _i, _p, _p, _p, _p]),
     "dsa_sparse_attn_decode": (_i, [_i, _i, _i, _i, _i, _f, _p, _p, _p, _i64, _p, _p, _p, _p, _sz, _p]),
     "dsa_small_workspace": (_sz, []),
     "dsa_indexer_scores": (_i, [_i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),

@@ -104,6 +104,17 @@ int ksteps_of(int dI, int dtype) { return (dI * (dtype == DSA_BF16 ? 2 : 1) + 31
 
 }  // namespace
 
+// Helpers shared with other translation units of the library (kernels.h).
+namespace dsa {
+void set_last_error(const char* msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+int device_sm_count() { return sm_count(); }
+uint64_t wait_timeout_ns() { return g_timeout_ns; }
+int encode_tensor_map(CUtensorMap* m, const void* base, int elem_bytes, uint64_t cols, uint64_t rows,
+                      uint32_t box_rows) {
+  return (int)make_tmap(m, base, elem_bytes, cols, rows, box_rows);
+}
+}  // namespace dsa
+
 extern "C" {
 
 const char* dsa_version(void) { return "dsa-b200 0.1 (sm_100a)"; }

@@ -89,4 +89,11 @@ cudaError_t launch_fill_f32(float* p, int64_t n, float v, cudaStream_t stream);
 cudaError_t launch_sparse_attn(const AttnArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_wait_selftest(DeviceStatus* status, uint64_t timeout_ns, cudaStream_t stream);
 
+// Host helpers implemented in api.cu.
+void set_last_error(const char* msg);                 // message returned by dsa_last_error()
+int device_sm_count();                                // SMs of the current device
+uint64_t wait_timeout_ns();                           // bound of every device-side wait
+int encode_tensor_map(CUtensorMap* m, const void* base, int elem_bytes, uint64_t cols, uint64_t rows,
+                      uint32_t box_rows);             // a dsa_status value
+
 }  // namespace dsa
