@@ -10,18 +10,28 @@
 // instruction whatever its shape, which caps an N = 16 product at ~1.4K
 // FLOP/clk/SM; warp-level mma.sync m16n8k16 sustains ~1.9K FLOP/clk/SM and
 // lets the 16 x Dqk query live in registers for the whole row, so it is used
-// here.  (Products with >= 128 rows per operand run on tcgen05 elsewhere.)
+// here.  The selected rows of one sequence sit in L2 (its latent tensor is a
+// few MB), so the gather is bounded by L2 -> SM bandwidth: one TMA bulk copy
+// per row, issued from four warps, sustains ~13 TB/s per GPU where 16-byte
+// cp.async from the same four warps reaches ~5.
 //
 // Work item = (query row, group of 16 heads); persistent grid, one CTA per SM.
 //   warps 0-3  producer: validate and compact the row's indices, then gather
-//              the selected latent rows 64 at a time with 16-byte cp.async into
-//              three 72 KB stages (128B-swizzled 64-column blocks);
+//              the selected latent rows 64 at a time (16 per warp, one bulk
+//              copy per row) into three stages of padded rows (1168-byte
+//              pitch: eight consecutive rows start in eight different bank
+//              groups, so ldmatrix needs no swizzle);
 //   warps 4-7  compute: the 16 x Dqk query as register-resident A fragments;
 //              warp w forms the logits of keys 16w..16w+15 of the chunk
-//              (S = Q C^T), the per-head running max / rescale (base-2
-//              exponent) is shared through shared memory, probabilities go to
-//              shared memory in bf16, and warp w accumulates O for value
-//              columns [128w, 128w+128) (O += P V) in fp32 registers.
+//              (S = Q C^T; even and odd k-steps in separate accumulators, each
+//              fragment loaded one step ahead of its MMAs), the per-head
+//              running max / rescale (base-2 exponent) is shared through shared
+//              memory, probabilities go to shared memory in bf16, and warp w
+//              accumulates O for value columns [128w, 128w+128) (O += P V) in
+//              fp32 registers.
+// Loop trip counts are fixed at the largest supported shape (Dqk 576, Dv
+// 512): columns past Dqk are zero in both operands (zeroed shared memory and
+// zero query fragments) and value columns past Dv are computed, not stored.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -33,16 +43,18 @@ namespace dsa {
 
 namespace {
 
-constexpr int kChunk = 64;            // keys per chunk
-constexpr int NH = 16;                // heads per work item (mma M)
+constexpr int kChunk = 64;                 // keys per chunk
+constexpr int NH = 16;                     // heads per work item (mma M)
 constexpr int kStages = 3;
-constexpr int kMaxCB = 9;             // 64-column blocks per row (Dqk <= 576)
-constexpr int kBlockBytes = kChunk * 128;
-constexpr int kStageBytes = kMaxCB * kBlockBytes;
+constexpr int kMaxDqk = 576;
+constexpr int kKsteps = kMaxDqk / 16;      // 36
+constexpr int kMaxDv = 512;
+constexpr int kPitch = kMaxDqk * 2 + 16;   // 1168 bytes per gathered row
+constexpr int kStageBytes = kChunk * kPitch;
 constexpr int kMaxK = 2048;
-constexpr int kMaxKsteps = kMaxCB * 4;  // 16-column steps of Dqk
 constexpr int kThreads = 256;
-constexpr int kProd = 128;             // producer threads (warps 0-3)
+constexpr int kProd = 128;                 // producer threads (warps 0-3)
+constexpr int kRowsPerWarp = kChunk / 4;   // rows copied per producer warp and chunk
 constexpr int kPBytes = NH * kChunk * 2;
 
 struct TokInfo {
@@ -60,62 +72,64 @@ __device__ __forceinline__ void row_geometry(const AttnArgs& a, int r, int64_t& 
   }
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
-__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-      : "r"(addr));
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
 }
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-      : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-      : "r"(addr));
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
 }
-__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                                         uint32_t b1) {
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+               "{%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
-// Byte offset of (row r, 16-byte chunk ch) inside a 128B-swizzled block.
+// Byte offset of (row r, 16-byte chunk ch) of the 128-byte-row P tile, chunks
+// XOR-swizzled by the row so the rows one ldmatrix reads fall in distinct
+// bank groups.
 __device__ __forceinline__ uint32_t swz(uint32_t r, uint32_t ch) { return r * 128u + ((ch ^ (r & 7u)) << 4); }
 
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  // the 128B swizzle here is address arithmetic (cp.async / ldmatrix), so
-  // 128-byte alignment of the blocks is enough
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  uint8_t* sC = base;                                                  // [3][9][64][128B]
-  uint8_t* sP = sC + kStages * kStageBytes;                            // [2][16 heads][64 keys] bf16, swizzled
-  uint16_t* sList = reinterpret_cast<uint16_t*>(sP + 2 * kPBytes);     // [kMaxK] compacted slot numbers
+  uint8_t* sC = base;                                                  // [3][64 rows][1168 B]
+  uint8_t* sP = sC + kStages * kStageBytes;                            // [16 heads][64 keys] bf16, swizzled
+  uint16_t* sList = reinterpret_cast<uint16_t*>(sP + kPBytes);         // [kMaxK] compacted slot numbers
   TokInfo* sTok = reinterpret_cast<TokInfo*>(sList + kMaxK);           // [2]
-  float* sMax = reinterpret_cast<float*>(sTok + 2);                    // [2][4 warps][16]
-  float* sSum = sMax + 2 * 4 * NH;                                     // [4][16]
+  float* sMax = reinterpret_cast<float*>(sTok + 2);                    // [4 warps][16]
+  float* sSum = sMax + 4 * NH;                                         // [4 warps][16]
   uint32_t* sWarpCnt = reinterpret_cast<uint32_t*>(sSum + 4 * NH);     // [4]
   uint32_t* sBcast = sWarpCnt + 4;                                     // [2]
   uint64_t* bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(sBcast + 2) + 7) & ~uintptr_t(7));
-  uint64_t* st_full = bars;               // [3] (producer threads, cp.async arrive)
-  uint64_t* st_empty = bars + kStages;    // [3] (4 compute warps)
+  uint64_t* st_full = bars;                  // [3] (4 producer warps + transaction bytes)
+  uint64_t* st_empty = bars + kStages;       // [3] (4 compute warps)
   uint64_t* tok_full = bars + 2 * kStages;   // [2]
   uint64_t* tok_empty = tok_full + 2;        // [2] (4 compute warps)
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(tok_empty + 2);
 
   const uint32_t warp = warp_id(), lane = lane_id();
+  // A row shorter than the pitch (Dqk < 576) leaves the tail of its slot as
+  // written here: zero, which the fixed-length loops then add nothing from.
+  for (uint32_t i = threadIdx.x; i < (uint32_t)(kStages * kStageBytes / 16); i += kThreads)
+    reinterpret_cast<uint4*>(sC)[i] = make_uint4(0u, 0u, 0u, 0u);
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&st_full[i], kProd);
+      mbar_init(&st_full[i], 4);
       mbar_init(&st_empty[i], 4);
     }
     for (int i = 0; i < 2; ++i) {
@@ -125,18 +139,24 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
     *abort_flag = 0u;
     mbar_fence_init();
   }
+  fence_proxy_async_smem();   // the zeros are ordered before the bulk copies
   __syncthreads();
   const WaitCtl ctl{abort_flag, a.timeout_ns, a.status};
   const int hg_count = (a.H + NH - 1) / NH;
   const int items = a.rows * hg_count;
-  const int CB = a.cb;
 
   if (warp < 4) {
     // ------------------------------------------------------------------ producer
+    // A failed wait only disables work: every producer thread still runs the
+    // same sequence of named barriers.
     const uint32_t pt = threadIdx.x;    // 0..127
+    const uint32_t row_bytes = (uint32_t)a.Dqk * 2u;
     int tslot = 0, stage = 0;
     uint32_t tphase = 0, sphase = 0;
     bool ok = true;
+    int last_phase[kStages];            // parity of this warp's last copies per stage, -1 none
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) last_phase[s] = -1;
     for (int item = blockIdx.x; item < items; item += gridDim.x) {
       const int r = item / hg_count;
       int64_t base_row;
@@ -146,14 +166,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
       // ---- compact the valid indices (slot order kept) into sList
       named_bar_sync(2, kProd);          // the previous row's list is no longer read
       constexpr int kPer = kMaxK / kProd;  // 16 slots per thread
-      int32_t pos[kPer];
       uint32_t vmask = 0;
 #pragma unroll
       for (int e = 0; e < kPer; ++e) {
         const int slot = (int)pt * kPer + e;
         const int p = slot < a.k ? __ldg(idx_row + slot) : -1;
         if (slot < a.k && (p < -1 || p >= len)) report_status(a.status, kStatusDeviceCheck, 0xA77Eu);
-        pos[e] = p;
         if (p >= 0 && p < len) vmask |= 1u << e;
       }
       const uint32_t mycnt = __popc(vmask);
@@ -184,62 +202,72 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
         mbar_arrive(&tok_full[tslot]);
       }
       if (++tslot == 2) { tslot = 0; tphase ^= 1u; }
-      // ---- gather 64 selected rows per chunk.  Thread pt copies 16-byte
-      // chunk (pt & 7) of every 128-byte block of rows (pt >> 3) + 16j,
-      // j = 0..3: eight consecutive lanes cover one 128-byte segment.  The
-      // four row numbers of the next chunk are fetched while waiting for a
-      // free stage, so no global load sits between the copies.
-      const uint32_t ch = pt & 7u, r0 = pt >> 3;
-      int64_t rows[4];
-      auto fetch_rows = [&](uint32_t c) {
-        const uint32_t nk = min((uint32_t)kChunk, nvalid - c * kChunk);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t rr = r0 + 16u * j;
-          rows[j] = base_row + __ldg(idx_row + sList[c * kChunk + (rr < nk ? rr : 0u)]);
-        }
+      // ---- gather: warp w copies rows 16w..16w+15 of every chunk, one bulk
+      // copy per row from lanes 0..15.  The row number of the next chunk is
+      // fetched while the stage is awaited.
+      const uint32_t rr = warp * kRowsPerWarp + (lane & (kRowsPerWarp - 1));
+      auto fetch_row = [&](uint32_t c) -> int64_t {
+        const uint32_t slot = c * kChunk + rr;
+        return (lane < (uint32_t)kRowsPerWarp && slot < nvalid) ? base_row + __ldg(idx_row + sList[slot]) : -1;
       };
-      if (nchunks > 0) fetch_rows(0);
+      int64_t row = nchunks > 0 ? fetch_row(0) : -1;
       for (uint32_t c = 0; c < nchunks; ++c) {
-        if (ok) ok = mbar_wait(&st_empty[stage], sphase ^ 1u, ctl, 0x2102);
+        int got = 1;
+        if (lane == 0 && ok) got = mbar_wait(&st_empty[stage], sphase ^ 1u, ctl, 0x2102) ? 1 : 0;
+        ok = ok && __shfl_sync(0xffffffffu, got, 0) != 0;
         if (ok) {
-          uint8_t* dst = sC + stage * kStageBytes;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t rr = r0 + 16u * j;
-            const uint16_t* src = a.latent + rows[j] * a.Dqk;
-            for (int cb = 0; cb < CB; ++cb) {
-              const int col = cb * 64 + (int)ch * 8;
-              const bool in = col < a.Dqk;
-              cp_async16(smem_u32(dst + cb * kBlockBytes + swz(rr, ch)), src + (in ? col : 0), in ? 16u : 0u);
-            }
-          }
+          const uint32_t mine = __ballot_sync(0xffffffffu, row >= 0);
+          if (lane == 0) mbar_arrive_expect_tx(&st_full[stage], (uint32_t)__popc(mine) * row_bytes);
+          __syncwarp();
+          if (row >= 0)
+            bulk_copy_g2s(smem_u32(sC + stage * kStageBytes + rr * kPitch), a.latent + row * a.Dqk, row_bytes,
+                          &st_full[stage]);
+          last_phase[stage] = (int)sphase;
         }
-        cp_async_arrive_noinc(&st_full[stage]);
         if (++stage == kStages) { stage = 0; sphase ^= 1u; }
-        if (c + 1 < nchunks) fetch_rows(c + 1);
+        if (c + 1 < nchunks) row = fetch_row(c + 1);
       }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (*abort_flag != 0u && lane == 0) {
+      // stopped early: give this warp's copies in flight time to land before
+      // the CTA exits (bounded; a stage another warp never armed stays open)
+#pragma unroll
+      for (int s = 0; s < kStages; ++s)
+        if (last_phase[s] >= 0) {
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(smem_u32(&st_full[s]), (uint32_t)last_phase[s]) &&
+                 globaltimer_ns() - t0 < a.timeout_ns) {
+          }
+        }
+    }
   } else {
     // ------------------------------------------------------------------ compute
     const uint32_t cw = warp - 4;                 // 0..3
     const uint32_t g = lane >> 2, c4 = lane & 3u; // mma fragment coordinates
-    const int ksteps = a.ksteps;
+    const uint32_t mi = lane >> 3;                // ldmatrix matrix this lane addresses
     int tslot = 0, stage = 0;
-    uint32_t tphase = 0, sphase = 0, pbuf = 0;
+    uint32_t tphase = 0, sphase = 0;
+    const uint32_t sC0 = smem_u32(sC), sP0 = smem_u32(sP);
+    // S: ldmatrix row = key 16cw + 8(mi>>1) + (lane&7), 8-column half (mi&1)
+    const uint32_t s_off = (cw * 16 + (mi >> 1) * 8 + (lane & 7u)) * kPitch + (mi & 1u) * 16;
+    // PV: key 8(mi&1) + (lane&7) of each 16-key step, value columns 128cw + 8(mi>>1)
+    const uint32_t v_off = ((mi & 1u) * 8 + (lane & 7u)) * kPitch + (cw * 128 + (mi >> 1) * 8) * 2;
+    // P: head (lane&15), 8-key half (lane>>4) of each 16-key step
+    const uint32_t p_row = lane & 15u, p_half = lane >> 4;
     for (int item = blockIdx.x; item < items; item += gridDim.x) {
       const int r = item / hg_count, hg = item - r * hg_count;
-      // queries of this head group -> A fragments (rows g, g+8; heads past H are zero)
-      uint32_t qa[kMaxKsteps][4];
+      // queries of this head group -> A fragments (rows g, g+8; heads past H
+      // and columns past Dqk are zero)
+      uint32_t qa[kKsteps][4];
       {
         const int h0 = hg * NH + (int)g, h1 = h0 + 8;
         const uint32_t* q0 = reinterpret_cast<const uint32_t*>(a.q + ((int64_t)r * a.H + h0) * a.Dqk);
         const uint32_t* q1 = reinterpret_cast<const uint32_t*>(a.q + ((int64_t)r * a.H + h1) * a.Dqk);
         const bool v0 = h0 < a.H, v1 = h1 < a.H;
+        const int kst = a.Dqk / 16;
 #pragma unroll
-        for (int ks = 0; ks < kMaxKsteps; ++ks) {
-          const bool in = ks < ksteps;
+        for (int ks = 0; ks < kKsteps; ++ks) {
+          const bool in = ks < kst;
           const int e = ks * 8 + (int)c4;           // 32-bit element index (2 bf16 each)
           qa[ks][0] = (in && v0) ? __ldg(q0 + e) : 0u;
           qa[ks][1] = (in && v1) ? __ldg(q1 + e) : 0u;
@@ -268,26 +296,35 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
       float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.0f, l_hi = 0.0f;   // heads g, g+8
 
       for (uint32_t c = 0; c < nchunks; ++c) {
+        // a failed wait has raised the abort flag; the chunk is then computed
+        // on stale data and the status word reports the failure
         (void)mbar_wait(&st_full[stage], sphase, ctl, 0x2302);
-        const uint32_t cbase = smem_u32(sC + stage * kStageBytes);
-        // ---- S = Q C^T for keys 16cw..16cw+15 (two n-tiles of 8 keys)
-        float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-        {
-          // ldmatrix x4: matrices (keys 0-7, dims 0-7), (keys 0-7, dims 8-15),
-          //                        (keys 8-15, dims 0-7), (keys 8-15, dims 8-15)
-          const uint32_t mi = lane >> 3;
-          const uint32_t key = cw * 16 + (mi >> 1) * 8 + (lane & 7);
-          const uint32_t dh = mi & 1;   // which 8-dim half of the 16-dim step
+        const uint32_t cbase = sC0 + stage * kStageBytes;
+        // ---- S = Q C^T for keys 16cw..16cw+15 (n-tiles 0, 1)
+        float sa[2][2][4];
 #pragma unroll
-          for (int ks = 0; ks < kMaxKsteps; ++ks) {
-            if (ks < ksteps) {
-              const uint32_t cb = (uint32_t)ks >> 2, ch = ((uint32_t)ks & 3u) * 2u + dh;
-              uint32_t b0, b1, b2, b3;
-              ldsm_x4(cbase + cb * kBlockBytes + swz(key, ch), b0, b1, b2, b3);
-              mma16816(s0, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
-              mma16816(s1, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) sa[i][j][0] = sa[i][j][1] = sa[i][j][2] = sa[i][j][3] = 0.0f;
+        {
+          uint32_t bc[4], bn[4];
+          ldsm_x4(cbase + s_off, bc);
+#pragma unroll
+          for (int ks = 0; ks < kKsteps; ++ks) {
+            if (ks + 1 < kKsteps) ldsm_x4(cbase + s_off + (ks + 1) * 32, bn);
+            mma16816(sa[ks & 1][0], qa[ks], bc[0], bc[1]);
+            mma16816(sa[ks & 1][1], qa[ks], bc[2], bc[3]);
+            if (ks + 1 < kKsteps) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) bc[i] = bn[i];
             }
           }
+        }
+        float s0[4], s1[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          s0[i] = sa[0][0][i] + sa[1][0][i];
+          s1[i] = sa[0][1][i] + sa[1][1][i];
         }
         // ---- mask, scale, chunk max per head
         const uint32_t kbase = c * kChunk + cw * 16 + 2 * c4;   // key of s0[0]
@@ -308,15 +345,16 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
         mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
         mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
         mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
-        float* smx = sMax + pbuf * 4 * NH;
         if (c4 == 0) {
-          smx[cw * NH + g] = mx_lo;
-          smx[cw * NH + g + 8] = mx_hi;
+          sMax[cw * NH + g] = mx_lo;
+          sMax[cw * NH + g + 8] = mx_hi;
         }
+        // barrier 1: every warp's chunk maxima are visible, and every warp has
+        // finished reading the previous chunk's P
         named_bar_sync(1, 128);
-        const float cm_lo = fmaxf(fmaxf(smx[g], smx[NH + g]), fmaxf(smx[2 * NH + g], smx[3 * NH + g]));
+        const float cm_lo = fmaxf(fmaxf(sMax[g], sMax[NH + g]), fmaxf(sMax[2 * NH + g], sMax[3 * NH + g]));
         const float cm_hi =
-            fmaxf(fmaxf(smx[g + 8], smx[NH + g + 8]), fmaxf(smx[2 * NH + g + 8], smx[3 * NH + g + 8]));
+            fmaxf(fmaxf(sMax[g + 8], sMax[NH + g + 8]), fmaxf(sMax[2 * NH + g + 8], sMax[3 * NH + g + 8]));
         const float mn_lo = fmaxf(m_lo, cm_lo), mn_hi = fmaxf(m_hi, cm_hi);
         const float al_lo = (m_lo == -INFINITY) ? 0.0f : exp2f(m_lo - mn_lo);
         const float al_hi = (m_hi == -INFINITY) ? 0.0f : exp2f(m_hi - mn_hi);
@@ -332,12 +370,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
         l_hi = l_hi * al_hi + (p02 + p03 + p12 + p13);
         // P[head][key] (bf16), row = head, 128 bytes per row, swizzled 16-byte chunks
         {
-          uint8_t* P = sP + pbuf * kPBytes;
           const uint32_t k0 = cw * 16 + 2 * c4;   // keys k0, k0+1 (n-tile 0) and k0+8, k0+9 (n-tile 1)
-          *reinterpret_cast<uint32_t*>(P + swz(g, k0 >> 3) + (k0 & 7) * 2) = pack_bf16(p00, p01);
-          *reinterpret_cast<uint32_t*>(P + swz(g + 8, k0 >> 3) + (k0 & 7) * 2) = pack_bf16(p02, p03);
-          *reinterpret_cast<uint32_t*>(P + swz(g, (k0 + 8) >> 3) + (k0 & 7) * 2) = pack_bf16(p10, p11);
-          *reinterpret_cast<uint32_t*>(P + swz(g + 8, (k0 + 8) >> 3) + (k0 & 7) * 2) = pack_bf16(p12, p13);
+          *reinterpret_cast<uint32_t*>(sP + swz(g, k0 >> 3) + (k0 & 7) * 2) = pack_bf16(p00, p01);
+          *reinterpret_cast<uint32_t*>(sP + swz(g + 8, k0 >> 3) + (k0 & 7) * 2) = pack_bf16(p02, p03);
+          *reinterpret_cast<uint32_t*>(sP + swz(g, (k0 + 8) >> 3) + (k0 & 7) * 2) = pack_bf16(p10, p11);
+          *reinterpret_cast<uint32_t*>(sP + swz(g + 8, (k0 + 8) >> 3) + (k0 & 7) * 2) = pack_bf16(p12, p13);
         }
         // rescale the running output
         if (al_lo != 1.0f || al_hi != 1.0f) {
@@ -349,25 +386,33 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
             o[j][3] *= al_hi;
           }
         }
+        // barrier 2: P is complete, and every warp has read this chunk's maxima
         named_bar_sync(1, 128);
-        // ---- O[:, 128cw .. 128cw+127] += P (16 x 64) V (64 x 128)
+        // ---- O[:, 128cw .. 128cw+127] += P (16 x 64) V (64 x 128); each
+        // fragment is loaded one step ahead of the MMAs that use it
         {
-          const uint32_t pbase = smem_u32(sP + pbuf * kPBytes);
-          const uint32_t mi = lane >> 3;
+          uint32_t pa[4], pn[4], vc[4], vn[4];
+          ldsm_x4(sP0 + swz(p_row, p_half), pa);
+          ldsm_x4_t(cbase + v_off, vc);
 #pragma unroll
           for (int kk = 0; kk < kChunk / 16; ++kk) {
-            uint32_t a0, a1, a2, a3;
-            // A = P rows (heads) 0-15, keys 16kk..16kk+15
-            ldsm_x4(pbase + swz(lane & 15u, (uint32_t)kk * 2u + (lane >> 4)), a0, a1, a2, a3);
-            const uint32_t key = kk * 16 + (mi & 1) * 8 + (lane & 7);
 #pragma unroll
             for (int j = 0; j < 16; j += 2) {
-              const uint32_t v0 = cw * 128 + j * 8 + (mi >> 1) * 8;   // value column of this matrix
-              if ((int)v0 < a.Dv) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_t(cbase + (v0 >> 6) * kBlockBytes + swz(key, (v0 & 63) >> 3), b0, b1, b2, b3);
-                mma16816(o[j], a0, a1, a2, a3, b0, b1);
-                mma16816(o[j + 1], a0, a1, a2, a3, b2, b3);
+              const bool last = kk == kChunk / 16 - 1 && j == 14;
+              if (j == 0 && kk + 1 < kChunk / 16) ldsm_x4(sP0 + swz(p_row, (uint32_t)(kk + 1) * 2u + p_half), pn);
+              if (!last) {
+                const int nkk = j == 14 ? kk + 1 : kk, nj = j == 14 ? 0 : j + 2;
+                ldsm_x4_t(cbase + v_off + nkk * 16 * kPitch + nj * 16, vn);
+              }
+              mma16816(o[j], pa, vc[0], vc[1]);
+              mma16816(o[j + 1], pa, vc[2], vc[3]);
+              if (!last) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) vc[i] = vn[i];
+                if (j == 14) {
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) pa[i] = pn[i];
+                }
               }
             }
           }
@@ -375,7 +420,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
         __syncwarp();
         if (lane == 0) mbar_arrive(&st_empty[stage]);
         if (++stage == kStages) { stage = 0; sphase ^= 1u; }
-        pbuf ^= 1u;
       }
       // ---- finish the row: O / l, log-sum-exp
       l_lo += __shfl_xor_sync(0xffffffffu, l_lo, 1);
@@ -418,13 +462,14 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
 // Host side
 // ---------------------------------------------------------------------------
 static size_t attn_smem() {
-  return 128 + (size_t)kStages * kStageBytes + 2 * kPBytes + kMaxK * 2 + 2 * sizeof(TokInfo) +
-         (2 * 4 * NH + 4 * NH) * 4 + 6 * 4 + 8 + (2 * kStages + 4) * 8 + 8;
+  return 128 + (size_t)kStages * kStageBytes + kPBytes + kMaxK * 2 + 2 * sizeof(TokInfo) + (2 * 4 * NH) * 4 +
+         6 * 4 + 8 + (2 * kStages + 4) * 8 + 8;
 }
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, int grid, cudaStream_t stream) {
   if (a.rows == 0) return cudaSuccess;
-  if (a.nh != NH || a.cb > kMaxCB || a.k > kMaxK || a.Dv > 512) return cudaErrorInvalidValue;
+  if (a.nh != NH || a.Dqk > kMaxDqk || a.Dqk % 16 != 0 || a.k > kMaxK || a.Dv > kMaxDv)
+    return cudaErrorInvalidValue;
   const size_t smem = attn_smem();
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
