@@ -73,7 +73,14 @@ uint64_t dsa_get_wait_timeout_ns(void);
 dsa_status dsa_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 /* Synchronise `stream`, return the device status recorded in `workspace`
  * (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_CHECK), store its detail word in
- * *detail if non-NULL, and clear it. */
+ * *detail if non-NULL, and clear it.  The first failure of a launch wins.
+ * Detail words: DSA_ERR_TIMEOUT -> the wait that gave up (0x1xxx indexer
+ * prefill, 0x2xxx sparse attention, 0x1xx..0x3xx indexer scan, 0x7e57
+ * self-test);
+ * DSA_ERR_DEVICE_CHECK -> 0xA77E an attention index outside [-1, L),
+ * 0x70E1 a top-k row longer than its matrix, 0x5e1ec6..0x5e1ec9 a selection
+ * whose candidate count broke its invariant (output slots may then hold
+ * any in-range position or -1). */
 dsa_status dsa_read_device_status(void* workspace, void* stream, uint32_t* detail);
 
 /* ------------------------------------------------------------------------

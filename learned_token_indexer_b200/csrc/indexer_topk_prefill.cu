@@ -361,7 +361,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           key = e.x;
           pos = e.y;
         };
-        group_find<128>(hist, kHistBins, (uint32_t)kk, true, sel, tid, bar_id);
+        // the filter keeps at least kk candidates, so the bin always exists;
+        // a miss is reported and the row is emitted from bin 0 (in bounds)
+        if (!group_find<128>(hist, kHistBins, (uint32_t)kk, true, sel, tid, bar_id) && tid == 0)
+          report_status(a.status, kStatusDeviceCheck, 0x5e1ec6u);
         const uint32_t b0 = sel.found_bin;
         const uint32_t need = (uint32_t)kk - sel.found_beyond;
         const uint32_t cnt = hist[b0];
@@ -372,7 +375,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         res.pos_hi = 0;
         if (need != cnt)
           res = group_refine<128, kHistBins>(get, m, res.lo, res.hi, need, (uint32_t)tok_t[g], hist, sel, tid,
-                                             bar_id);
+                                             bar_id, a.status);
         const int64_t row = (int64_t)blk.b * a.nq + blk.t0 + st;
         group_emit<128>(get, m, res, kk, a.k, a.idx_out + row * a.k,
                         a.score_out ? a.score_out + row * a.k : nullptr, sel, tid, bar_id, a.status);

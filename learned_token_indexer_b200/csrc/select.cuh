@@ -45,10 +45,19 @@ struct SelectShared {
 // Find the bin where the running count over `nbins` bins, traversed from the
 // top (from_top) or from the bottom, first reaches `need` (1 <= need <= total).
 // Result: sh.found_bin, sh.found_beyond = count strictly before it in
-// traversal order.  All NT threads call it; it ends with a barrier.
+// traversal order.  All NT threads call it; it ends with a barrier.  Returns
+// false (and leaves bin 0, nothing before it) when the bins hold fewer than
+// `need` entries -- a broken caller invariant; callers report it and stop.
+// Callers read the result before their next barrier and call again only
+// after one.
 template <int NT>
-__device__ __forceinline__ void group_find(const uint32_t* hist, int nbins, uint32_t need, bool from_top,
+__device__ __forceinline__ bool group_find(const uint32_t* hist, int nbins, uint32_t need, bool from_top,
                                            SelectShared<NT>& sh, uint32_t tid, uint32_t bar_id) {
+  constexpr uint32_t kNotFound = 0xFFFFFFFFu;
+  if (tid == 0) {
+    sh.found_bin = kNotFound;
+    sh.found_beyond = 0u;
+  }
   const int per = (nbins + NT - 1) / NT;
   const int i0 = (int)tid * per;
   uint32_t local = 0;
@@ -78,6 +87,11 @@ __device__ __forceinline__ void group_find(const uint32_t* hist, int nbins, uint
     }
   }
   named_bar_sync(bar_id, NT);
+  if (sh.found_bin != kNotFound) return true;
+  named_bar_sync(bar_id, NT);   // every thread has seen the miss before it is cleared
+  if (tid == 0) sh.found_bin = 0u;
+  named_bar_sync(bar_id, NT);
+  return false;
 }
 
 // Refine a cut-off inside [lo, hi] (need >= 1 entries to take there, entries
@@ -85,7 +99,8 @@ __device__ __forceinline__ void group_find(const uint32_t* hist, int nbins, uint
 // `hist` is NBINS uint32 of shared scratch owned by the group.
 template <int NT, int NBINS, typename Get>
 __device__ SelectResult group_refine(Get get, int m, uint32_t lo, uint32_t hi, uint32_t need, uint32_t pos_max,
-                                     uint32_t* hist, SelectShared<NT>& sh, uint32_t tid, uint32_t bar_id) {
+                                     uint32_t* hist, SelectShared<NT>& sh, uint32_t tid, uint32_t bar_id,
+                                     DeviceStatus* status) {
   SelectResult r;
   r.key_all_in = 0;
   r.pos_hi = 0;
@@ -110,7 +125,13 @@ __device__ SelectResult group_refine(Get get, int m, uint32_t lo, uint32_t hi, u
         if (i0 + u * NT < m && key[u] >= lo && key[u] <= hi) atomicAdd(&hist[(key[u] >> s) - base], 1u);
     }
     named_bar_sync(bar_id, NT);
-    group_find<NT>(hist, nb, need, true, sh, tid, bar_id);
+    if (!group_find<NT>(hist, nb, need, true, sh, tid, bar_id)) {
+      if (tid == 0) report_status(status, kStatusDeviceCheck, 0x5e1ec8u);
+      r.lo = lo;
+      r.hi = hi;
+      r.key_all_in = 1;
+      return r;
+    }
     const uint32_t d = sh.found_bin;
     const uint32_t cnt = hist[d];
     need -= sh.found_beyond;
@@ -151,7 +172,10 @@ __device__ SelectResult group_refine(Get get, int m, uint32_t lo, uint32_t hi, u
           atomicAdd(&hist[(pos[u] >> s) - base], 1u);
     }
     named_bar_sync(bar_id, NT);
-    group_find<NT>(hist, nb, need, false, sh, tid, bar_id);
+    if (!group_find<NT>(hist, nb, need, false, sh, tid, bar_id)) {
+      if (tid == 0) report_status(status, kStatusDeviceCheck, 0x5e1ec9u);
+      break;
+    }
     const uint32_t d = sh.found_bin;
     const uint32_t cnt = hist[d];
     need -= sh.found_beyond;

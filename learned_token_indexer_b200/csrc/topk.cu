@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRow
   r.pos_hi = 0;
   if (kk > 0 && kk < len)
     r = group_refine<kRowThreads, kRowBins>(get, len, 0u, 0xFFFFFFFFu, (uint32_t)kk, (uint32_t)(len - 1), hist, sh,
-                                             tid, 0);
+                                             tid, 0, a.status);
   else if (kk == len && len > 0)
     r.lo = 0u;   // every entry is selected
   group_emit<kRowThreads>(get, kk > 0 ? len : 0, r, kk, a.k, idx_row, val_row, sh, tid, 0, a.status);
