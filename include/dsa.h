@@ -15,8 +15,8 @@
  *    (a cudaStream_t passed as void*; NULL = legacy default stream).
  *  - bf16 tensors hold raw bfloat16 bit patterns; FP8 tensors hold E4M3
  *    ("fn", max 448) codes, one byte each, with one positive fp32 scale per
- *    token (the dequantised value is code * scale, §2 "quantised indexer key
- *    cache with scales").
+ *    token (the dequantised value is code * scale; §2 keeps the indexer key
+ *    cache quantised, with its scales).
  *  - Base pointers of the indexer operands (qI, kI) must be 16-byte aligned
  *    (they are read with TMA); other tensors need their natural alignment.
  *  - Positions are 0-based.  A query at absolute position t may select keys
