@@ -55,6 +55,48 @@ __device__ __forceinline__ void bin_key_range(uint32_t b, uint32_t& lo, uint32_t
   hi = (z << 21) | 0x1FFFFFu;
 }
 
+// Raise a token's floor from its histogram (one warp): the bin where the
+// running count of accepted scores, from the top bin down, first reaches k
+// (at least k accepted scores lie in that bin or above, so nothing in a lower
+// bin can enter the top k).  Lane l sums bins [512 - 16(l+1), 512 - 16l).
+__device__ __forceinline__ void raise_floor(const uint32_t* hist, uint32_t k, uint32_t* floor_key, uint32_t lane) {
+  constexpr int kPerLane = kHistBins / 32;
+  const int b0 = kHistBins - kPerLane * ((int)lane + 1);
+  uint32_t h[kPerLane];
+  uint32_t local = 0;
+#pragma unroll
+  for (int j = 0; j < kPerLane; ++j) {
+    h[j] = hist[b0 + j];
+    local += h[j];
+  }
+  uint32_t incl = local;   // count from the top bin down to this lane's lowest bin
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= (uint32_t)o) incl += v;
+  }
+  const uint32_t reach = __ballot_sync(0xffffffffu, incl >= k);
+  if (reach == 0u) return;   // fewer than k accepted so far
+  const uint32_t L = (uint32_t)(__ffs(reach) - 1);
+  if (lane == L) {
+    // highest bin of this lane's range where the running count reaches k
+    // (no early exit, so h stays in registers)
+    uint32_t run = incl - local;
+    int f = b0;
+    bool found = false;
+#pragma unroll
+    for (int j = kPerLane - 1; j >= 0; --j) {
+      run += h[j];
+      const bool hit = !found && run >= k;
+      f = hit ? b0 + j : f;
+      found = found || hit;
+    }
+    uint32_t lo, hi;
+    bin_key_range((uint32_t)f, lo, hi);
+    if (lo > *floor_key) *floor_key = lo;
+  }
+}
+
 struct Block {
   int b, t0;      // sequence, first local query row
   int nvalid;     // valid tokens in the block (<= 8)
@@ -104,10 +146,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint8_t* sQ = sK + STAGES * kKBytes;
   float* sW = reinterpret_cast<float*>(sQ + 2 * kQGroupBytes);            // [8][HI]
   uint32_t* sHist = reinterpret_cast<uint32_t*>(sW + kQB * HI);           // [8][512]
-  uint32_t* sCount = sHist + kQB * kHistBins;                             // [8]
-  uint32_t* sFloor = sCount + kQB;                                        // [8]
-  uint32_t* sBelow = sFloor + kQB;                                        // [8]
-  SelectShared<128>* sSel = reinterpret_cast<SelectShared<128>*>(sBelow + kQB);  // [4]
+  uint32_t* sCnt = sHist + kQB * kHistBins;                               // [8][4 warps]
+  uint32_t* sFloorKey = sCnt + kQB * 4;                                   // [8]
+  SelectShared<128>* sSel = reinterpret_cast<SelectShared<128>*>(sFloorKey + kQB);  // [4]
   uint64_t* bars = reinterpret_cast<uint64_t*>(
       (reinterpret_cast<uintptr_t>(sSel + 4) + 7) & ~uintptr_t(7));
   uint64_t* k_full = bars;
@@ -246,7 +287,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint32_t wg = (warp - 2) >> 2;                  // 0..3
     const uint32_t tid = (warp - 2 - 4 * wg) * 32 + lane; // 0..127 inside the warpgroup
     const uint32_t bar_id = 2 + wg;
-    const uint32_t lane_grp = (warp & 3u) * 32u;
+    const uint32_t quarter = warp & 3u;                   // TMEM lane quarter of this warp
+    const uint32_t lane_grp = quarter * 32u;
     const uint32_t key_in_tile = lane_grp + lane;
     SelectShared<128>& sel = sSel[wg];
     uint32_t aphase[2] = {0u, 0u};
@@ -267,11 +309,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const int g = i / kHistBins;
         sHist[(kTA * g + wg) * kHistBins + (i - g * kHistBins)] = 0u;
       }
-      if (tid < 2u) {
-        sCount[kTA * tid + wg] = 0u;
-        sFloor[kTA * tid + wg] = 0u;
-        sBelow[kTA * tid + wg] = 0u;
-      }
+      if (tid < 2u) sFloorKey[kTA * tid + wg] = 0u;   // key 0: every score passes
       for (int i = (int)tid; i < 2 * HI; i += 128) {
         const int g = i / HI, h = i - g * HI;
         const int li = blk.t0 + kTA * g + (int)wg;
@@ -285,65 +323,53 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       named_bar_sync(bar_id, 128);
       const int nt_max = max(blk.nt[0], blk.nt[1]);
-      uint2* cand_tok[2];
+      // accepted (key, position) pairs: this warp's sub-buffer of each token
+      // (warp q of the group sees keys with s mod 128 in [32q, 32q + 32))
+      uint2* cand_w[2];
+      uint32_t cnt[2] = {0u, 0u};
 #pragma unroll
       for (int g = 0; g < 2; ++g)
-        cand_tok[g] = a.cand + ((int64_t)blockIdx.x * kQB + kTA * g + wg) * a.cand_cap;
+        cand_w[g] = a.cand + ((int64_t)blockIdx.x * kQB + kTA * g + wg) * a.cand_cap + quarter * (a.cand_cap / 4);
       for (int t = 0; t < nt_max; ++t) {
         const int s = t * kTileKeys + (int)key_in_tile;
         float ks = 1.0f;
         if (FP8 && ok) ks = (s < a.kv_len) ? a.k_scale[(int64_t)blk.b * a.kv_len + s] : 0.0f;
-        float score[2] = {0.0f, 0.0f};
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
           if (t >= blk.nt[g]) continue;
           const bool got = ok && mbar_wait(&acc_full[g], aphase[g], ctl, 0x1301);
           ok = __all_sync(0xffffffffu, got);
           aphase[g] ^= 1u;
-          if (ok) {
-            tc_fence_after();
-            float sc[1];
-            group_head_sums<HI, 1>(tmem_base + (lane_grp << 16) + g * N + wg * HI, sW + (kTA * g + wg) * HI, sc,
-                                   &acc_empty[g], lane);
-            score[g] = FP8 ? sc[0] * ks : sc[0];
-          }
-        }
-        named_bar_sync(bar_id, 128);     // previous tile's floor update is visible
-        if (ok) {
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            if (t >= blk.nt[g]) continue;
-            const int st = kTA * g + (int)wg;
-            const uint32_t key = float_to_key(score[g]);
+          if (!ok) continue;
+          tc_fence_after();
+          float sc[1];
+          group_head_sums<HI, 1>(tmem_base + (lane_grp << 16) + g * N + wg * HI, sW + (kTA * g + wg) * HI, sc,
+                                 &acc_empty[g], lane);
+          const float score = FP8 ? sc[0] * ks : sc[0];
+          // streaming filter: a key below the token's floor cannot be in its
+          // top k (the floor only rises; another warp may raise it meanwhile)
+          const int st = kTA * g + (int)wg;
+          const uint32_t key = float_to_key(score);
+          const uint32_t floor_key = *reinterpret_cast<volatile const uint32_t*>(&sFloorKey[st]);
+          const bool acc = tok_valid[g] && s <= tok_t[g] && key >= floor_key;
+          const uint32_t mask = __ballot_sync(0xffffffffu, acc);
+          if (acc) {
+            cand_w[g][cnt[g] + __popc(mask & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)s);
+            // histogram of accepted scores, one atomic per distinct bin of the warp
             const uint32_t bin = score_bin(key);
-            const bool acc = tok_valid[g] && s <= tok_t[g] && bin >= sFloor[st];
-            const uint32_t mask = __ballot_sync(0xffffffffu, acc);
-            if (mask) {
-              uint32_t slot0 = 0;
-              if (lane == 0) slot0 = atomicAdd(&sCount[st], (uint32_t)__popc(mask));
-              slot0 = __shfl_sync(0xffffffffu, slot0, 0);
-              if (acc) {
-                const uint32_t slot = slot0 + __popc(mask & ((1u << lane) - 1u));
-                cand_tok[g][slot] = make_uint2(key, (uint32_t)s);
-                atomicAdd(&sHist[st * kHistBins + bin], 1u);
-              }
-            }
+            const uint32_t peers = __match_any_sync(mask, bin);
+            if (lane == (uint32_t)(__ffs(peers) - 1)) atomicAdd(&sHist[st * kHistBins + bin], (uint32_t)__popc(peers));
           }
-        }
-        named_bar_sync(bar_id, 128);     // this tile's appends are complete
-        if (ok && tid < 2u && t < blk.nt[tid]) {
-          const int st = kTA * (int)tid + (int)wg;
-          const uint32_t* h = sHist + st * kHistBins;
-          const uint32_t c = sCount[st];
-          uint32_t fl = sFloor[st], bl = sBelow[st];
-          while (fl < kLastBin && c - bl - h[fl] >= (uint32_t)a.k) {
-            bl += h[fl];
-            ++fl;
-          }
-          sFloor[st] = fl;
-          sBelow[st] = bl;
+          cnt[g] += (uint32_t)__popc(mask);
+          // raise the floor (warp q = g of the group, every tile): the bin
+          // where the count of accepted scores from the top first reaches k
+          if (quarter == (uint32_t)g) raise_floor(sHist + st * kHistBins, (uint32_t)a.k, &sFloorKey[st], lane);
         }
       }
+      // per-warp candidate counts for the select
+#pragma unroll
+      for (int g = 0; g < 2; ++g)
+        if (lane == 0) sCnt[(kTA * g + wg) * 4 + quarter] = cnt[g];
       named_bar_sync(bar_id, 128);
       if (tid == 0) sel.aborted = *abort_flag;
       named_bar_sync(bar_id, 128);
@@ -353,11 +379,28 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (!tok_valid[g] || blk.nt[g] == 0) continue;
         const int st = kTA * g + (int)wg;
         const int kk = min(a.k, tok_t[g] + 1);
-        const int m = (int)sCount[st];
+        const uint32_t c0 = sCnt[st * 4], c1 = sCnt[st * 4 + 1], c2 = sCnt[st * 4 + 2], c3 = sCnt[st * 4 + 3];
+        const int m = (int)(c0 + c1 + c2 + c3);
         uint32_t* hist = sHist + st * kHistBins;
-        const uint2* buf = cand_tok[g];
-        auto get = [buf](int i, uint32_t& key, uint32_t& pos) {
-          const uint2 e = buf[i];
+        const uint2* buf = a.cand + ((int64_t)blockIdx.x * kQB + st) * a.cand_cap;
+        const int64_t sub = a.cand_cap / 4;
+        // entry i of the token's candidates: the four warp sub-buffers in order
+        auto get = [=](int i, uint32_t& key, uint32_t& pos) {
+          uint32_t off = (uint32_t)i;
+          int q = 0;
+          if (off >= c0) {
+            off -= c0;
+            q = 1;
+            if (off >= c1) {
+              off -= c1;
+              q = 2;
+              if (off >= c2) {
+                off -= c2;
+                q = 3;
+              }
+            }
+          }
+          const uint2 e = buf[q * sub + off];
           key = e.x;
           pos = e.y;
         };
@@ -398,7 +441,7 @@ struct PrefillConfig {
   static constexpr int N = kTA * HI;
   static constexpr int kQBytes = 2 * N * KB * kSwizzleBytes;
   static constexpr int kKBytes = kTileKeys * KB * kSwizzleBytes;
-  static constexpr int kFixed = 1024 /*align*/ + kQBytes + kQB * HI * 4 + kQB * kHistBins * 4 + 3 * kQB * 4 +
+  static constexpr int kFixed = 1024 /*align*/ + kQBytes + kQB * HI * 4 + kQB * kHistBins * 4 + 5 * kQB * 4 +
                                 4 * (int)sizeof(SelectShared<128>) + 8 + 16 * 8 + 16;
   static constexpr int kBudget = 227 * 1024;
   static constexpr int kStagesFit = (kBudget - kFixed) / kKBytes;
