@@ -70,7 +70,7 @@ def kernel_source_hash(files):
 
 KERNEL_SOURCES = {
     "indexer_topk_prefill": ["indexer_topk_prefill.cu", "indexer_common.cuh", "select.cuh", "sm100.cuh"],
-    "sparse_attn": ["sparse_attn.cu"],
+    "sparse_attn": ["sparse_attn.cu", "sm100.cuh"],
     "indexer_scan": ["indexer_scan.cu", "indexer_common.cuh", "sm100.cuh"],
     "topk_rows": ["topk.cu", "select.cuh"],
 }
