@@ -22,6 +22,7 @@ the same workload on the host cores.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -404,6 +405,28 @@ def workload_label(w: W.Workload):
     return (f"prefill B={w.B} n={w.n} HI={w.HI} dI={w.dI} k={w.k} {dt}{ch}; attn H={w.H} latent {w.Dqk}/{w.Dv}")
 
 
+def max_over_ranks(x: float, device) -> float:
+    """Max of a per-rank number over all ranks (identity without a process
+    group): every multi-rank duration in the JSON line is the slowest rank's."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return x
+    if torch.distributed.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_workload(w, rank: int):
+    """Each rank draws its own batch of the same workload (weak scaling)."""
+    return w if rank == 0 else dataclasses.replace(w, seed=w.seed + 7919 * rank)
+
+
+def job_throughput(world: int, units_per_rank: int, ms_per_step: float) -> float:
+    """Units every rank processed in one step, over the slowest rank's step time."""
+    return world * units_per_rank / (ms_per_step * 1e-3)
+
+
 def run_b200(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -419,7 +442,7 @@ def run_b200(args):
         build()
     if world > 1:
         torch.distributed.barrier()
-    w = W.ALL[args.workload]
+    w = rank_workload(W.ALL[args.workload], rank)
     run = DecodeRun(w, dev) if w.kind == "decode" else PrefillRun(w, dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
@@ -439,19 +462,12 @@ def run_b200(args):
     clocks = sampler.stop()
     run.ws_idx.check()
     run.ws_att.check()
-    ms = float(np.mean(step_ms))
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(float(np.mean(step_ms)), dev)
     e2e = None
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_e2e(run, max(3, min(10, args.steps)))
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": world * run.rows() / (e2e_ms * 1e-3), "unit": METRIC[w.kind if w.kind == "decode" else "prefill"][1],
+        e2e_ms = max_over_ranks(e2e_ms, dev)
+        e2e = {"value": job_throughput(world, run.rows(), e2e_ms), "unit": METRIC[w.kind if w.kind == "decode" else "prefill"][1],
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
     if world > 1:
         torch.distributed.barrier()
@@ -489,7 +505,7 @@ def run_b200(args):
     roof["peak_source"] = f"{peak_src} ({'fp8 = 2 x measured bf16' if (w.fp8 and roof['bound'] == 'tensor' and dom == names[0]) else 'burst bf16 / copy bandwidth'})"
     metric, unit = METRIC["decode" if w.kind == "decode" else "prefill"]
     line = {
-        "metric": metric, "value": world * run.rows() / (ms * 1e-3), "unit": unit, "n_gpus": world,
+        "metric": metric, "value": job_throughput(world, run.rows(), ms), "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8-e4m3 indexer / bf16 attention, fp32 accumulate" if w.fp8 else "bf16 in, fp32 accumulate",
