@@ -9,33 +9,39 @@
 // logits product is 16 x keys x Dqk.  tcgen05.mma costs >= ~46 cycles per
 // instruction whatever its shape, which caps an N = 16 product at ~1.4K
 // FLOP/clk/SM; warp-level mma.sync m16n8k16 sustains ~1.9K FLOP/clk/SM and
-// lets the 16 x Dqk query live in registers for the whole row, so it is used
-// here.  The selected rows of one sequence sit in L2 (its latent tensor is a
-// few MB), so the gather is bounded by L2 -> SM bandwidth: one TMA bulk copy
-// per row, issued from four warps, sustains ~13 TB/s per GPU where 16-byte
+// lets the query live in registers for the whole row, so it is used here.
+// The selected rows of one sequence sit in L2 (its latent tensor is a few
+// MB), so the gather is bounded by L2 -> SM bandwidth: one TMA bulk copy per
+// row, issued from four warps, sustains ~13 TB/s per GPU where 16-byte
 // cp.async from the same four warps reaches ~5.
 //
 // Work item = (query row, group of 16 heads); persistent grid, one CTA per SM,
-// three warpgroups that work on consecutive chunks of 64 selected rows at once:
-//   WG0 producer: validate and compact the row's indices, prefetch the row's
-//       queries into L2, then gather the selected latent rows (16 per warp,
-//       one bulk copy per row) into three stages of padded rows (1168-byte
-//       pitch: eight consecutive rows start in eight different bank groups,
-//       so ldmatrix needs no swizzle);
-//   WG1 logits + softmax: the 16 x Dqk query as register-resident A
-//       fragments; warp w forms the logits of keys 16w..16w+15 of chunk c
-//       (S = Q C^T; even and odd k-steps in separate accumulators, each
-//       fragment loaded one step ahead of its MMAs), the warps agree on the
-//       per-head running max through shared memory (base-2 exponent), then
-//       hand the bf16 probabilities P and the per-head rescale factor to WG2;
-//   WG2 values: warp w accumulates O for value columns [128w, 128w+128)
-//       (O = alpha O + P V) in fp32 registers for chunk c - 1 while WG1 works
-//       on chunk c, and writes the normalised output at the end of the row.
-// Registers are rebalanced between the warpgroups (setmaxnreg): the logits
-// group holds the query fragments, the value group the output accumulators.
-// Loop trip counts are fixed at the largest supported shape (Dqk 576, Dv
-// 512): columns past Dqk are zero in both operands (zeroed shared memory and
-// zero query fragments) and value columns past Dv are computed, not stored.
+// four warpgroups working on consecutive chunks of 64 selected rows at once:
+//   WG0-1 producers: validate the row's indices into per-32-slot validity
+//       masks and prefix counts, prefetch the row's queries into L2, then
+//       gather the selected latent rows (8 per warp, one bulk copy per row;
+//       bulk copies from one warp issue one after another) into three
+//       stages of padded rows (1168-byte pitch: eight consecutive rows start
+//       in eight different bank groups, so ldmatrix needs no swizzle);
+//   WG2 logits: warp w owns keys 16w..16w+15 of every chunk.  It forms their
+//       logits (S = Q C^T, the 16 x Dqk query as register-resident A
+//       fragments), keeps its own running max per head (base-2 exponent) and
+//       emits bf16 P = 2^(S - M_w) relative to that max, with M_w, into one of
+//       two hand-off slots.  The warps never wait for one another inside a row;
+//       they combine their softmax denominators once, at the row's end;
+//   WG3 values: warp w accumulates O for value columns [128w, 128w+128)
+//       (O += P V) in fp32 registers against a reference max R per head: it
+//       raises R to the largest M_w of the chunk, rescales O by 2^(R_old - R),
+//       and multiplies each logits warp's 16-key block of P by 2^(M_w - R)
+//       before its MMAs.  At the row's end R equals the row max, so O / L is
+//       the softmax-weighted sum.
+// In the MMA loops even and odd k-steps go to separate accumulators and every
+// fragment is requested two steps ahead of its MMAs; the next row's queries
+// are requested as soon as the current row's last logits are formed.
+// Registers are rebalanced between the warpgroups (setmaxnreg).  Loop trip
+// counts are fixed at the largest supported shape (Dqk 576, Dv 512): columns
+// past Dqk are zero in both operands (zeroed shared memory and zero query
+// fragments) and value columns past Dv are computed, not stored.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -56,28 +62,33 @@ constexpr int kMaxDv = 512;
 constexpr int kPitch = kMaxDqk * 2 + 16;   // 1168 bytes per gathered row
 constexpr int kStageBytes = kChunk * kPitch;
 constexpr int kMaxK = 2048;
-constexpr int kThreads = 384;
-constexpr int kProd = 128;                 // producer threads (warps 0-3)
-constexpr int kRowsPerWarp = kChunk / 4;   // rows copied per producer warp and chunk
+constexpr int kBlocks = kMaxK / 32;        // 32-slot validity blocks of an index row
+constexpr int kThreads = 512;
+constexpr int kProdWarps = 8;              // producer warps 0-7 (two warpgroups)
+constexpr int kProd = kProdWarps * 32;
+constexpr int kRowsPerWarp = kChunk / kProdWarps;   // rows copied per producer warp and chunk
 constexpr int kPBytes = NH * kChunk * 2;
-// per-thread register budgets after the split; their sum over the three
-// warpgroups equals the launch allocation (168 per thread)
-constexpr int kLaunchRegs = 168;
-constexpr int kRegsProd = 56, kRegsLogits = 240, kRegsValues = 208;
-static_assert(kRegsProd + kRegsLogits + kRegsValues == 3 * kLaunchRegs, "register split must match the launch");
+constexpr int kSlots = 2;                  // logits -> values hand-off slots
+// per-thread register budgets after the split; their sum over the four
+// warpgroups equals the launch allocation (128 per thread)
+constexpr int kLaunchRegs = 128;
+constexpr int kRegsProd = 56, kRegsLogits = 232, kRegsValues = 168;
+static_assert(2 * kRegsProd + kRegsLogits + kRegsValues == 4 * kLaunchRegs, "register split must match the launch");
+
+// named barriers (0 is __syncthreads)
+constexpr uint32_t kBarLogits = 1, kBarProd = 2;
 
 struct TokInfo {
   uint32_t nvalid;
   uint32_t nchunks;
 };
 
-// Logits group -> value group, one per chunk (single slot, guarded by the
-// p_full / p_empty barriers together with P).
+// Logits group -> value group, one per chunk, with the chunk's P.
 struct Msg {
-  int32_t item;        // work item of the chunk; -1: no more work
-  uint32_t flags;      // bit 0: first chunk of the item, bit 1: last chunk
-  float alpha[NH];     // factor on the running output before this chunk
-  float inv_l[NH];     // last chunk: 1 / softmax denominator (0 if empty)
+  int32_t item;          // work item of the chunk; -1: no more work
+  uint32_t flags;        // bit 0: first chunk of the item, bit 1: last chunk
+  float m[4][NH];        // running max of each logits warp after this chunk (-inf: none yet)
+  float inv_l[NH];       // last chunk: 1 / softmax denominator at the row max (0 if empty)
 };
 constexpr uint32_t kFirst = 1u, kLast = 2u;
 
@@ -127,10 +138,78 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
+// lane-wise bf16 product of two packed pairs, rounded to nearest
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t x, uint32_t y) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(x), "r"(y));
+  return d;
+}
 // Byte offset of (row r, 16-byte chunk ch) of the 128-byte-row P tile, chunks
 // XOR-swizzled by the row so the rows one ldmatrix reads fall in distinct
 // bank groups.
 __device__ __forceinline__ uint32_t swz(uint32_t r, uint32_t ch) { return r * 128u + ((ch ^ (r & 7u)) << 4); }
+
+// Position of the (rank+1)-th set bit of m (rank < popc(m)).
+__device__ __forceinline__ uint32_t nth_set_bit(uint32_t m, uint32_t rank) {
+  uint32_t pos = 0;
+#pragma unroll
+  for (uint32_t w = 16; w > 0; w >>= 1) {
+    const uint32_t low = __popc(m & ((1u << w) - 1u));
+    if (rank >= low) {
+      rank -= low;
+      m >>= w;
+      pos += w;
+    }
+  }
+  return pos;
+}
+
+// Query fragments of one item (rows g, g+8 of the head group; heads past H
+// and columns past Dqk are zero).
+__device__ __forceinline__ void load_q(const AttnArgs& a, int hg_count, int item, uint32_t g, uint32_t c4,
+                                       uint32_t (&qa)[kKsteps][4]) {
+  const int r = item / hg_count, hg = item - r * hg_count;
+  const int h0 = hg * NH + (int)g, h1 = h0 + 8;
+  const uint32_t* q0 = reinterpret_cast<const uint32_t*>(a.q + ((int64_t)r * a.H + h0) * a.Dqk);
+  const uint32_t* q1 = reinterpret_cast<const uint32_t*>(a.q + ((int64_t)r * a.H + h1) * a.Dqk);
+  const bool v0 = h0 < a.H, v1 = h1 < a.H;
+  const int kst = a.Dqk / 16;
+#pragma unroll
+  for (int ks = 0; ks < kKsteps; ++ks) {
+    const bool in = ks < kst;
+    const int e = ks * 8 + (int)c4;           // 32-bit element index (2 bf16 each)
+    qa[ks][0] = (in && v0) ? __ldg(q0 + e) : 0u;
+    qa[ks][1] = (in && v1) ? __ldg(q1 + e) : 0u;
+    qa[ks][2] = (in && v0) ? __ldg(q0 + e + 4) : 0u;
+    qa[ks][3] = (in && v1) ? __ldg(q1 + e + 4) : 0u;
+  }
+}
+
+// Logits of keys 16w..16w+15: s0 = n-tile 0 (keys +0..7), s1 = n-tile 1
+// (keys +8..15).
+__device__ __forceinline__ void logits(uint32_t row_addr, const uint32_t (&qa)[kKsteps][4], float (&s0)[4],
+                                       float (&s1)[4]) {
+  float sa[2][2][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) sa[i][j][0] = sa[i][j][1] = sa[i][j][2] = sa[i][j][3] = 0.0f;
+  // fragments of step i live in b[i % 3], requested two steps ahead
+  uint32_t b[3][4];
+  ldsm_x4(row_addr, b[0]);
+  ldsm_x4(row_addr + 32, b[1]);
+#pragma unroll
+  for (int i = 0; i < kKsteps; ++i) {
+    if (i + 2 < kKsteps) ldsm_x4(row_addr + (i + 2) * 32, b[(i + 2) % 3]);
+    mma16816(sa[i & 1][0], qa[i], b[i % 3][0], b[i % 3][1]);
+    mma16816(sa[i & 1][1], qa[i], b[i % 3][2], b[i % 3][3]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    s0[i] = sa[0][0][i] + sa[1][0][i];
+    s1[i] = sa[0][1][i] + sa[1][1][i];
+  }
+}
 
 // Output rows of heads g and g+8 of an item, value columns 128w + 8j + 2c4.
 __device__ __forceinline__ void store_out(const AttnArgs& a, int r, int hg, uint32_t w, uint32_t g, uint32_t c4,
@@ -156,22 +235,22 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   uint8_t* sC = base;                                                  // [3][64 rows][1168 B]
-  uint8_t* sP = sC + kStages * kStageBytes;                            // [16 heads][64 keys] bf16, swizzled
-  uint16_t* sList = reinterpret_cast<uint16_t*>(sP + kPBytes);         // [kMaxK] compacted slot numbers
-  TokInfo* sTok = reinterpret_cast<TokInfo*>(sList + kMaxK);           // [2]
-  float* sMax = reinterpret_cast<float*>(sTok + 2);                    // [2 parities][4 warps][16]
-  float* sSum = sMax + 2 * 4 * NH;                                     // [4 warps][16]
-  Msg* sMsg = reinterpret_cast<Msg*>(sSum + 4 * NH);
-  uint32_t* sWarpCnt = reinterpret_cast<uint32_t*>(sMsg + 1);          // [4]
-  uint32_t* sBcast = sWarpCnt + 4;                                     // [2]
+  uint8_t* sP = sC + kStages * kStageBytes;                            // [2 slots][16 heads][64 keys] bf16
+  Msg* sMsg = reinterpret_cast<Msg*>(sP + kSlots * kPBytes);           // [2 slots]
+  uint32_t* sMask = reinterpret_cast<uint32_t*>(sMsg + kSlots);        // [64] validity of 32-slot blocks
+  uint32_t* sPre = sMask + kBlocks;                                    // [65] valid entries before each block
+  TokInfo* sTok = reinterpret_cast<TokInfo*>(sPre + kBlocks + 1);      // [2]
+  float* sFin = reinterpret_cast<float*>(sTok + 2);                    // [2][4 warps][16] row-end max, sum
+  uint32_t* sWarpCnt = reinterpret_cast<uint32_t*>(sFin + 2 * 4 * NH); // [8]
+  uint32_t* sBcast = sWarpCnt + kProdWarps;                            // [2]
   uint64_t* bars = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(sBcast + 2) + 7) & ~uintptr_t(7));
-  uint64_t* st_full = bars;                  // [3] (4 producer warps + transaction bytes)
+  uint64_t* st_full = bars;                  // [3] (8 producer warps + transaction bytes)
   uint64_t* st_empty = bars + kStages;       // [3] (4 value warps)
   uint64_t* tok_full = bars + 2 * kStages;   // [2] (1 producer thread)
   uint64_t* tok_empty = tok_full + 2;        // [2] (4 logits warps)
-  uint64_t* p_full = tok_empty + 2;          // (128 logits threads)
-  uint64_t* p_empty = p_full + 1;            // (4 value warps)
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(p_empty + 1);
+  uint64_t* p_full = tok_empty + 2;          // [2] (128 logits threads)
+  uint64_t* p_empty = p_full + kSlots;       // [2] (4 value warps)
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(p_empty + kSlots);
 
   const uint32_t warp = warp_id(), lane = lane_id();
   // A row shorter than the pitch (Dqk < 576) leaves the tail of its slot as
@@ -180,15 +259,17 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
     reinterpret_cast<uint4*>(sC)[i] = make_uint4(0u, 0u, 0u, 0u);
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&st_full[i], 4);
+      mbar_init(&st_full[i], kProdWarps);
       mbar_init(&st_empty[i], 4);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tok_full[i], 1);
       mbar_init(&tok_empty[i], 4);
     }
-    mbar_init(p_full, 128);
-    mbar_init(p_empty, 4);
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(&p_full[i], 128);
+      mbar_init(&p_empty[i], 4);
+    }
     *abort_flag = 0u;
     mbar_fence_init();
   }
@@ -197,8 +278,11 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
   const WaitCtl ctl{abort_flag, a.timeout_ns, a.status};
   const int hg_count = (a.H + NH - 1) / NH;
   const int items = a.rows * hg_count;
+  const uint32_t g = lane >> 2, c4 = lane & 3u;   // mma fragment coordinates
+  const uint32_t mi = lane >> 3;                  // ldmatrix matrix this lane addresses
+  const uint32_t sC0 = smem_u32(sC), sP0 = smem_u32(sP);
 
-  if (warp < 4) {
+  if (warp < (uint32_t)kProdWarps) {
     // ================================================================ producer
     // A failed wait only disables work: every producer thread still runs the
     // same sequence of named barriers.
@@ -223,9 +307,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
         const int lines = (nh * a.Dqk * 2 + 127) / 128;
         for (int i = (int)pt; i < lines; i += kProd) prefetch_l2(q0 + (int64_t)i * 128);
       }
-      // ---- compact the valid indices (slot order kept) into sList
-      named_bar_sync(2, kProd);          // the previous row's list is no longer read
-      constexpr int kPer = kMaxK / kProd;  // 16 slots per thread
+      // ---- validity masks: thread pt owns slots [8pt, 8pt + 8); four threads
+      // (consecutive lanes) make one 32-slot block
+      named_bar_sync(kBarProd, kProd);   // the previous row's masks are no longer read
+      constexpr int kPer = kMaxK / kProd;
       uint32_t vmask = 0;
 #pragma unroll
       for (int e = 0; e < kPer; ++e) {
@@ -241,19 +326,25 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
         const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= (uint32_t)o) incl += v;
       }
+      static_assert(kPer == 8, "four threads per 32-slot block");
+      const uint32_t m1 = __shfl_down_sync(0xffffffffu, vmask, 1);
+      const uint32_t m2 = __shfl_down_sync(0xffffffffu, vmask, 2);
+      const uint32_t m3 = __shfl_down_sync(0xffffffffu, vmask, 3);
       if (lane == 31) sWarpCnt[warp] = incl;
-      named_bar_sync(2, kProd);
+      named_bar_sync(kBarProd, kProd);
       uint32_t off = incl - mycnt, nvalid = 0;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
+      for (int w = 0; w < kProdWarps; ++w) {
         const uint32_t c = sWarpCnt[w];
         if ((uint32_t)w < warp) off += c;
         nvalid += c;
       }
-#pragma unroll
-      for (int e = 0; e < kPer; ++e)
-        if (vmask & (1u << e)) sList[off++] = (uint16_t)(pt * kPer + e);
-      named_bar_sync(2, kProd);
+      if ((pt & 3u) == 0u) {
+        sMask[pt >> 2] = vmask | (m1 << 8) | (m2 << 16) | (m3 << 24);
+        sPre[pt >> 2] = off;
+      }
+      if (pt == 0) sPre[kBlocks] = nvalid;
+      named_bar_sync(kBarProd, kProd);
       const uint32_t nchunks = (nvalid + kChunk - 1) / kChunk;
       if (pt == 0) {
         if (ok) ok = mbar_wait(&tok_empty[tslot], tphase ^ 1u, ctl, 0x2101);
@@ -262,13 +353,23 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
         mbar_arrive(&tok_full[tslot]);
       }
       if (++tslot == 2) { tslot = 0; tphase ^= 1u; }
-      // ---- gather: warp w copies rows 16w..16w+15 of every chunk, one bulk
-      // copy per row from lanes 0..15.  The row number of the next chunk is
+      // ---- gather: warp w copies rows 8w..8w+7 of every chunk, one bulk
+      // copy per row from lanes 0..7 (bulk copies from one warp are issued one
+      // after another, so eight warps share the issuing).  The j-th valid slot is found from the
+      // prefix counts and the block's mask; the next chunk's row number is
       // fetched while the stage is awaited.
       const uint32_t rr = warp * kRowsPerWarp + (lane & (kRowsPerWarp - 1));
       auto fetch_row = [&](uint32_t c) -> int64_t {
-        const uint32_t slot = c * kChunk + rr;
-        return (lane < (uint32_t)kRowsPerWarp && slot < nvalid) ? base_row + __ldg(idx_row + sList[slot]) : -1;
+        const uint32_t j = c * kChunk + rr;
+        if (lane >= (uint32_t)kRowsPerWarp || j >= nvalid) return -1;
+        uint32_t lo = 0, hi = kBlocks;   // sPre[lo] <= j < sPre[hi]
+#pragma unroll
+        for (int it = 0; it < 6; ++it) {
+          const uint32_t mid = (lo + hi) >> 1;
+          if (sPre[mid] <= j) lo = mid; else hi = mid;
+        }
+        const uint32_t slot = lo * 32u + nth_set_bit(sMask[lo], j - sPre[lo]);
+        return base_row + __ldg(idx_row + slot);
       };
       int64_t row = nchunks > 0 ? fetch_row(0) : -1;
       for (uint32_t c = 0; c < nchunks; ++c) {
@@ -300,54 +401,32 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
           }
         }
     }
-  } else if (warp < 8) {
+  } else if (warp < (uint32_t)kProdWarps + 4) {
     // ================================================================ logits
-    // Every logits thread runs the same sequence of named barriers (chunk
-    // counts are broadcast); a failed wait only leaves stale data behind.
+    // Every thread of the group runs the same sequence of named barriers
+    // (chunk counts are broadcast); a failed wait only leaves stale data.
     regs_inc<kRegsLogits>();
-    const uint32_t sw = warp - 4;                 // 0..3
-    const uint32_t g = lane >> 2, c4 = lane & 3u; // mma fragment coordinates
-    const uint32_t mi = lane >> 3;                // ldmatrix matrix this lane addresses
-    int tslot = 0, stage = 0;
-    uint32_t tphase = 0, sphase = 0, pphase = 0;
-    const uint32_t sC0 = smem_u32(sC);
-    // ldmatrix row = key 16sw + 8(mi>>1) + (lane&7), 8-column half (mi&1)
+    const uint32_t sw = warp - kProdWarps;
     const uint32_t s_off = (sw * 16 + (mi >> 1) * 8 + (lane & 7u)) * kPitch + (mi & 1u) * 16;
-    uint32_t parity = 0;                          // chunk parity (sMax double buffer)
+    int tslot = 0, stage = 0, slot = 0;
+    uint32_t tphase = 0, sphase = 0, pphase = 0;
+    uint32_t qa[kKsteps][4];
+    if ((int)blockIdx.x < items) load_q(a, hg_count, blockIdx.x, g, c4, qa);
     for (int item = blockIdx.x; item < items; item += gridDim.x) {
       const int r = item / hg_count, hg = item - r * hg_count;
-      // queries of this head group -> A fragments (rows g, g+8; heads past H
-      // and columns past Dqk are zero)
-      uint32_t qa[kKsteps][4];
-      {
-        const int h0 = hg * NH + (int)g, h1 = h0 + 8;
-        const uint32_t* q0 = reinterpret_cast<const uint32_t*>(a.q + ((int64_t)r * a.H + h0) * a.Dqk);
-        const uint32_t* q1 = reinterpret_cast<const uint32_t*>(a.q + ((int64_t)r * a.H + h1) * a.Dqk);
-        const bool v0 = h0 < a.H, v1 = h1 < a.H;
-        const int kst = a.Dqk / 16;
-#pragma unroll
-        for (int ks = 0; ks < kKsteps; ++ks) {
-          const bool in = ks < kst;
-          const int e = ks * 8 + (int)c4;           // 32-bit element index (2 bf16 each)
-          qa[ks][0] = (in && v0) ? __ldg(q0 + e) : 0u;
-          qa[ks][1] = (in && v1) ? __ldg(q1 + e) : 0u;
-          qa[ks][2] = (in && v0) ? __ldg(q0 + e + 4) : 0u;
-          qa[ks][3] = (in && v1) ? __ldg(q1 + e + 4) : 0u;
-        }
-      }
+      const int next_item = item + (int)gridDim.x;
       (void)mbar_wait(&tok_full[tslot], tphase, ctl, 0x2301);
-      named_bar_sync(1, 128);
-      if (threadIdx.x == kProd) {
+      named_bar_sync(kBarLogits, 128);
+      if (threadIdx.x == (uint32_t)kProd) {
         const bool ab = *abort_flag != 0u;
         sBcast[0] = ab ? 0u : sTok[tslot].nvalid;
         sBcast[1] = ab ? 0u : sTok[tslot].nchunks;
       }
-      named_bar_sync(1, 128);
+      named_bar_sync(kBarLogits, 128);
       const uint32_t nvalid = sBcast[0], nchunks = sBcast[1];
       __syncwarp();
       if (lane == 0) mbar_arrive(&tok_empty[tslot]);
       if (++tslot == 2) { tslot = 0; tphase ^= 1u; }
-
       if (nchunks == 0) {
         // nothing selected: zero output, log-sum-exp -inf
         float z[16][4];
@@ -359,40 +438,19 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
           if (h_lo < a.H) a.lse[(int64_t)r * a.H + h_lo] = -INFINITY;
           if (h_hi < a.H) a.lse[(int64_t)r * a.H + h_hi] = -INFINITY;
         }
+        if (next_item < items) load_q(a, hg_count, next_item, g, c4, qa);
         continue;
       }
-      float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.0f, l_hi = 0.0f;   // heads g, g+8
+      // this warp's running max and denominator of heads g, g+8
+      float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.0f, l_hi = 0.0f;
       for (uint32_t c = 0; c < nchunks; ++c) {
         (void)mbar_wait(&st_full[stage], sphase, ctl, 0x2302);
-        const uint32_t cbase = sC0 + stage * kStageBytes;
-        // ---- S = Q C^T for keys 16sw..16sw+15 (n-tiles 0, 1)
-        float sa[2][2][4];
-#pragma unroll
-        for (int i = 0; i < 2; ++i)
-#pragma unroll
-          for (int j = 0; j < 2; ++j) sa[i][j][0] = sa[i][j][1] = sa[i][j][2] = sa[i][j][3] = 0.0f;
-        {
-          uint32_t bc[4], bn[4];
-          ldsm_x4(cbase + s_off, bc);
-#pragma unroll
-          for (int ks = 0; ks < kKsteps; ++ks) {
-            if (ks + 1 < kKsteps) ldsm_x4(cbase + s_off + (ks + 1) * 32, bn);
-            mma16816(sa[ks & 1][0], qa[ks], bc[0], bc[1]);
-            mma16816(sa[ks & 1][1], qa[ks], bc[2], bc[3]);
-            if (ks + 1 < kKsteps) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) bc[i] = bn[i];
-            }
-          }
-        }
         float s0[4], s1[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          s0[i] = sa[0][0][i] + sa[1][0][i];
-          s1[i] = sa[0][1][i] + sa[1][1][i];
-        }
+        logits(sC0 + stage * kStageBytes + s_off, qa, s0, s1);
         if (++stage == kStages) { stage = 0; sphase ^= 1u; }
-        // ---- mask, scale, chunk max per head
+        const bool last = c + 1 == nchunks;
+        if (last && next_item < items) load_q(a, hg_count, next_item, g, c4, qa);
+        // ---- mask, scale, running max of this warp's keys
         const uint32_t kbase = c * kChunk + sw * 16 + 2 * c4;   // key of s0[0]
         const bool k00 = kbase < nvalid, k01 = kbase + 1 < nvalid, k10 = kbase + 8 < nvalid,
                    k11 = kbase + 9 < nvalid;
@@ -411,17 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
         mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, 2));
         mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 1));
         mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, 2));
-        float* smx = sMax + parity * 4 * NH;
-        if (c4 == 0) {
-          smx[sw * NH + g] = mx_lo;
-          smx[sw * NH + g + 8] = mx_hi;
-        }
-        named_bar_sync(1, 128);   // every warp's chunk maxima are visible
-        const float cm_lo = fmaxf(fmaxf(smx[g], smx[NH + g]), fmaxf(smx[2 * NH + g], smx[3 * NH + g]));
-        const float cm_hi =
-            fmaxf(fmaxf(smx[g + 8], smx[NH + g + 8]), fmaxf(smx[2 * NH + g + 8], smx[3 * NH + g + 8]));
-        parity ^= 1u;
-        const float mn_lo = fmaxf(m_lo, cm_lo), mn_hi = fmaxf(m_hi, cm_hi);
+        const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
         const float al_lo = (m_lo == -INFINITY) ? 0.0f : exp2f(m_lo - mn_lo);
         const float al_hi = (m_hi == -INFINITY) ? 0.0f : exp2f(m_hi - mn_hi);
         m_lo = mn_lo;
@@ -434,68 +482,83 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
         const float p12 = exp2f(s1[2] - mu_hi), p13 = exp2f(s1[3] - mu_hi);
         l_lo = l_lo * al_lo + (p00 + p01 + p10 + p11);
         l_hi = l_hi * al_hi + (p02 + p03 + p12 + p13);
-        const bool last = c + 1 == nchunks;
         float il_lo = 0.0f, il_hi = 0.0f;
         if (last) {
-          // softmax denominators of the row: quad sums, then across warps
+          // the row's denominators at the row max: every warp's (max, sum)
           float t_lo = l_lo, t_hi = l_hi;
           t_lo += __shfl_xor_sync(0xffffffffu, t_lo, 1);
           t_lo += __shfl_xor_sync(0xffffffffu, t_lo, 2);
           t_hi += __shfl_xor_sync(0xffffffffu, t_hi, 1);
           t_hi += __shfl_xor_sync(0xffffffffu, t_hi, 2);
+          float* fm = sFin;            // [4][16] maxima
+          float* fl = sFin + 4 * NH;   // [4][16] sums
           if (c4 == 0) {
-            sSum[sw * NH + g] = t_lo;
-            sSum[sw * NH + g + 8] = t_hi;
+            fm[sw * NH + g] = m_lo;
+            fm[sw * NH + g + 8] = m_hi;
+            fl[sw * NH + g] = t_lo;
+            fl[sw * NH + g + 8] = t_hi;
           }
-          named_bar_sync(1, 128);
-          const float L_lo = sSum[g] + sSum[NH + g] + sSum[2 * NH + g] + sSum[3 * NH + g];
-          const float L_hi = sSum[g + 8] + sSum[NH + g + 8] + sSum[2 * NH + g + 8] + sSum[3 * NH + g + 8];
+          named_bar_sync(kBarLogits, 128);
+          float R_lo = -INFINITY, R_hi = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            R_lo = fmaxf(R_lo, fm[w * NH + g]);
+            R_hi = fmaxf(R_hi, fm[w * NH + g + 8]);
+          }
+          float L_lo = 0.0f, L_hi = 0.0f;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const float ml = fm[w * NH + g], mh = fm[w * NH + g + 8];
+            if (ml != -INFINITY) L_lo += fl[w * NH + g] * exp2f(ml - R_lo);
+            if (mh != -INFINITY) L_hi += fl[w * NH + g + 8] * exp2f(mh - R_hi);
+          }
+          named_bar_sync(kBarLogits, 128);   // sFin is reused by the next row
           il_lo = L_lo > 0.0f ? 1.0f / L_lo : 0.0f;
           il_hi = L_hi > 0.0f ? 1.0f / L_hi : 0.0f;
           if (a.lse && sw == 0 && c4 == 0) {
             const float ln2 = 0.69314718055994531f;
             const int h_lo = hg * NH + (int)g, h_hi = h_lo + 8;
-            if (h_lo < a.H) a.lse[(int64_t)r * a.H + h_lo] = L_lo > 0.0f ? (m_lo + log2f(L_lo)) * ln2 : -INFINITY;
-            if (h_hi < a.H) a.lse[(int64_t)r * a.H + h_hi] = L_hi > 0.0f ? (m_hi + log2f(L_hi)) * ln2 : -INFINITY;
+            if (h_lo < a.H) a.lse[(int64_t)r * a.H + h_lo] = L_lo > 0.0f ? (R_lo + log2f(L_lo)) * ln2 : -INFINITY;
+            if (h_hi < a.H) a.lse[(int64_t)r * a.H + h_hi] = L_hi > 0.0f ? (R_hi + log2f(L_hi)) * ln2 : -INFINITY;
           }
         }
-        // ---- hand P and the factors to the value group once it has taken
-        // the previous chunk's
-        (void)mbar_wait(p_empty, pphase ^ 1u, ctl, 0x2303);
+        // ---- hand P (relative to this warp's max) and the max over
+        (void)mbar_wait(&p_empty[slot], pphase ^ 1u, ctl, 0x2303);
+        uint8_t* P = sP + slot * kPBytes;
+        Msg* msg = sMsg + slot;
         {
           const uint32_t k0 = sw * 16 + 2 * c4;   // keys k0, k0+1 (n-tile 0) and k0+8, k0+9 (n-tile 1)
-          *reinterpret_cast<uint32_t*>(sP + swz(g, k0 >> 3) + (k0 & 7) * 2) = pack_bf16(p00, p01);
-          *reinterpret_cast<uint32_t*>(sP + swz(g + 8, k0 >> 3) + (k0 & 7) * 2) = pack_bf16(p02, p03);
-          *reinterpret_cast<uint32_t*>(sP + swz(g, (k0 + 8) >> 3) + (k0 & 7) * 2) = pack_bf16(p10, p11);
-          *reinterpret_cast<uint32_t*>(sP + swz(g + 8, (k0 + 8) >> 3) + (k0 & 7) * 2) = pack_bf16(p12, p13);
+          *reinterpret_cast<uint32_t*>(P + swz(g, k0 >> 3) + (k0 & 7) * 2) = pack_bf16(p00, p01);
+          *reinterpret_cast<uint32_t*>(P + swz(g + 8, k0 >> 3) + (k0 & 7) * 2) = pack_bf16(p02, p03);
+          *reinterpret_cast<uint32_t*>(P + swz(g, (k0 + 8) >> 3) + (k0 & 7) * 2) = pack_bf16(p10, p11);
+          *reinterpret_cast<uint32_t*>(P + swz(g + 8, (k0 + 8) >> 3) + (k0 & 7) * 2) = pack_bf16(p12, p13);
         }
-        if (sw == 0 && c4 == 0) {
-          sMsg->alpha[g] = al_lo;
-          sMsg->alpha[g + 8] = al_hi;
-          sMsg->inv_l[g] = il_lo;
-          sMsg->inv_l[g + 8] = il_hi;
+        if (c4 == 0) {
+          msg->m[sw][g] = m_lo;
+          msg->m[sw][g + 8] = m_hi;
+          if (sw == 0) {
+            msg->inv_l[g] = il_lo;
+            msg->inv_l[g + 8] = il_hi;
+          }
         }
         if (sw == 0 && lane == 0) {
-          sMsg->item = item;
-          sMsg->flags = (c == 0 ? kFirst : 0u) | (last ? kLast : 0u);
+          msg->item = item;
+          msg->flags = (c == 0 ? kFirst : 0u) | (last ? kLast : 0u);
         }
-        mbar_arrive(p_full);
-        pphase ^= 1u;
+        mbar_arrive(&p_full[slot]);
+        if (++slot == kSlots) { slot = 0; pphase ^= 1u; }
       }
     }
     // no more work for the value group
-    (void)mbar_wait(p_empty, pphase ^ 1u, ctl, 0x2304);
-    if (sw == 0 && lane == 0) sMsg->item = -1;
-    mbar_arrive(p_full);
+    (void)mbar_wait(&p_empty[slot], pphase ^ 1u, ctl, 0x2304);
+    if (sw == 0 && lane == 0) sMsg[slot].item = -1;
+    mbar_arrive(&p_full[slot]);
   } else {
     // ================================================================ values
     regs_inc<kRegsValues>();
-    const uint32_t vw = warp - 8;                 // 0..3
-    const uint32_t g = lane >> 2, c4 = lane & 3u;
-    const uint32_t mi = lane >> 3;
-    int stage = 0;
+    const uint32_t vw = warp - kProdWarps - 4;
+    int stage = 0, slot = 0;
     uint32_t sphase = 0, pphase = 0;
-    const uint32_t sC0 = smem_u32(sC), sP0 = smem_u32(sP);
     // key 8(mi&1) + (lane&7) of each 16-key step, value columns 128vw + 8(mi>>1)
     const uint32_t v_off = ((mi & 1u) * 8 + (lane & 7u)) * kPitch + (vw * 128 + (mi >> 1) * 8) * 2;
     // P: head (lane&15), 8-key half (lane>>4) of each 16-key step
@@ -503,65 +566,91 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
     float o[16][4];
 #pragma unroll
     for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
+    float R_lo = -INFINITY, R_hi = -INFINITY;    // reference max of heads g, g+8
     for (;;) {
-      if (!mbar_wait(p_full, pphase, ctl, 0x2401)) break;
-      pphase ^= 1u;
-      const int item = sMsg->item;
+      if (!mbar_wait(&p_full[slot], pphase, ctl, 0x2401)) break;
+      const Msg* msg = sMsg + slot;
+      const int item = msg->item;
       if (item < 0) break;
-      const uint32_t flags = sMsg->flags;
-      const float al_lo = sMsg->alpha[g], al_hi = sMsg->alpha[g + 8];
-      const float il_lo = sMsg->inv_l[g], il_hi = sMsg->inv_l[g + 8];
+      const uint32_t flags = msg->flags;
+      float wm_lo[4], wm_hi[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        wm_lo[w] = msg->m[w][g];
+        wm_hi[w] = msg->m[w][g + 8];
+      }
+      const float il_lo = msg->inv_l[g], il_hi = msg->inv_l[g + 8];
+      // raise the reference to the chunk's largest warp max, rescale O
+      float rn_lo = fmaxf(fmaxf(wm_lo[0], wm_lo[1]), fmaxf(wm_lo[2], wm_lo[3]));
+      float rn_hi = fmaxf(fmaxf(wm_hi[0], wm_hi[1]), fmaxf(wm_hi[2], wm_hi[3]));
       if (flags & kFirst) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
-      } else if (al_lo != 1.0f || al_hi != 1.0f) {
+      } else {
+        rn_lo = fmaxf(rn_lo, R_lo);
+        rn_hi = fmaxf(rn_hi, R_hi);
+        const float al_lo = exp2f(R_lo - rn_lo), al_hi = exp2f(R_hi - rn_hi);
+        if (al_lo != 1.0f || al_hi != 1.0f) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          o[j][0] *= al_lo;
-          o[j][1] *= al_lo;
-          o[j][2] *= al_hi;
-          o[j][3] *= al_hi;
+          for (int j = 0; j < 16; ++j) {
+            o[j][0] *= al_lo;
+            o[j][1] *= al_lo;
+            o[j][2] *= al_hi;
+            o[j][3] *= al_hi;
+          }
         }
+      }
+      R_lo = rn_lo;
+      R_hi = rn_hi;
+      // factor of each logits warp's block: 2^(M_w - R) (0 while M_w = -inf),
+      // as a bf16 pair per head row
+      uint32_t f_lo[4], f_hi[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float a_lo = wm_lo[w] == -INFINITY ? 0.0f : exp2f(wm_lo[w] - R_lo);
+        const float a_hi = wm_hi[w] == -INFINITY ? 0.0f : exp2f(wm_hi[w] - R_hi);
+        f_lo[w] = pack_bf16(a_lo, a_lo);
+        f_hi[w] = pack_bf16(a_hi, a_hi);
       }
       // the stage's bytes landed before the logits group released P (this
       // wait returns at once; it only makes the ordering explicit)
       (void)mbar_wait(&st_full[stage], sphase, ctl, 0x2402);
       const uint32_t cbase = sC0 + stage * kStageBytes;
-      // ---- O[:, 128vw .. 128vw+127] += P (16 x 64) V (64 x 128); each
-      // fragment is loaded one step ahead of the MMAs that use it
+      const uint32_t pbase = sP0 + slot * kPBytes;
+      // ---- O[:, 128vw .. 128vw+127] += P (16 x 64) V (64 x 128)
       {
-        uint32_t pa[4], pn[4], vc[4], vn[4];
-        ldsm_x4(sP0 + swz(p_row, p_half), pa);
-        ldsm_x4_t(cbase + v_off, vc);
+        // step t = 8 kk + j/2 covers keys 16kk.. (logits warp kk) and value
+        // columns 16(j/2)..; its fragments live in vb[t % 3], requested two
+        // steps ahead; the scaled P fragments of step kk live in pa[kk & 1]
+        constexpr int kSteps = (kChunk / 16) * 8;
+        auto v_addr = [&](int t) { return cbase + v_off + (t >> 3) * 16 * kPitch + (t & 7) * 32; };
+        auto load_p = [&](int kk, uint32_t (&p)[4]) {
+          ldsm_x4(pbase + swz(p_row, (uint32_t)kk * 2u + p_half), p);
+          p[0] = mul_bf16x2(p[0], f_lo[kk]);
+          p[1] = mul_bf16x2(p[1], f_hi[kk]);
+          p[2] = mul_bf16x2(p[2], f_lo[kk]);
+          p[3] = mul_bf16x2(p[3], f_hi[kk]);
+        };
+        uint32_t pa[2][4], vb[3][4];
+        load_p(0, pa[0]);
+        ldsm_x4_t(v_addr(0), vb[0]);
+        ldsm_x4_t(v_addr(1), vb[1]);
 #pragma unroll
-        for (int kk = 0; kk < kChunk / 16; ++kk) {
-#pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            const bool lastf = kk == kChunk / 16 - 1 && j == 14;
-            if (j == 0 && kk + 1 < kChunk / 16) ldsm_x4(sP0 + swz(p_row, (uint32_t)(kk + 1) * 2u + p_half), pn);
-            if (!lastf) {
-              const int nkk = j == 14 ? kk + 1 : kk, nj = j == 14 ? 0 : j + 2;
-              ldsm_x4_t(cbase + v_off + nkk * 16 * kPitch + nj * 16, vn);
-            }
-            mma16816(o[j], pa, vc[0], vc[1]);
-            mma16816(o[j + 1], pa, vc[2], vc[3]);
-            if (!lastf) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) vc[i] = vn[i];
-              if (j == 14) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) pa[i] = pn[i];
-              }
-            }
-          }
+        for (int t = 0; t < kSteps; ++t) {
+          const int kk = t >> 3, j = (t & 7) * 2;
+          if (j == 0 && kk + 1 < kChunk / 16) load_p(kk + 1, pa[(kk + 1) & 1]);
+          if (t + 2 < kSteps) ldsm_x4_t(v_addr(t + 2), vb[(t + 2) % 3]);
+          mma16816(o[j], pa[kk & 1], vb[t % 3][0], vb[t % 3][1]);
+          mma16816(o[j + 1], pa[kk & 1], vb[t % 3][2], vb[t % 3][3]);
         }
       }
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&st_empty[stage]);
-        mbar_arrive(p_empty);
+        mbar_arrive(&p_empty[slot]);
       }
       if (++stage == kStages) { stage = 0; sphase ^= 1u; }
+      if (++slot == kSlots) { slot = 0; pphase ^= 1u; }
       if (flags & kLast) {
         const int r = item / hg_count, hg = item - r * hg_count;
         store_out(a, r, hg, vw, g, c4, o, il_lo, il_hi);
@@ -575,8 +664,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_attn_kernel(const AttnArgs
 // Host side
 // ---------------------------------------------------------------------------
 static size_t attn_smem() {
-  return 128 + (size_t)kStages * kStageBytes + kPBytes + kMaxK * 2 + 2 * sizeof(TokInfo) + (3 * 4 * NH) * 4 +
-         sizeof(Msg) + 6 * 4 + 8 + (2 * kStages + 6) * 8 + 8;
+  return 128 + (size_t)kStages * kStageBytes + kSlots * (kPBytes + sizeof(Msg)) + (2 * kBlocks + 1) * 4 +
+         2 * sizeof(TokInfo) + 2 * 4 * NH * 4 + (kProdWarps + 2) * 4 + 8 + (2 * kStages + 4 + 2 * kSlots) * 8 + 8;
 }
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, int grid, cudaStream_t stream) {
