@@ -164,7 +164,8 @@ size_t dsa_sparse_attn_workspace(void) { return kHeader; }
 size_t dsa_indexer_topk_prefill_workspace(int B, int nq, int kv_len, int HI, int dI, int k, int dtype) {
   (void)B; (void)nq; (void)HI; (void)dI; (void)k; (void)dtype;
   const size_t cap = round_up((size_t)(kv_len > 0 ? kv_len : 1), 128);   // 4 warp sub-buffers of cap / 4
-  return kHeader + (size_t)sm_count() * dsa::prefill_block_tokens() * cap * sizeof(uint2);
+  // candidates of the 8 tokens of a block, then one cut-off scratch per epilogue group
+  return kHeader + (size_t)sm_count() * (dsa::prefill_block_tokens() + 4) * cap * sizeof(uint2);
 }
 
 dsa_status dsa_indexer_topk_prefill(int B, int nq, int q_offset, int kv_len, int HI, int dI, int k, int dtype,
@@ -212,6 +213,7 @@ dsa_status dsa_indexer_topk_prefill(int B, int nq, int q_offset, int kv_len, int
   a.score_out = score_out;
   a.cand = reinterpret_cast<uint2*>(static_cast<char*>(workspace) + kHeader);
   a.cand_cap = (int64_t)round_up((size_t)kv_len, 128);
+  a.bnd = a.cand + (int64_t)sm_count() * dsa::prefill_block_tokens() * a.cand_cap;
   a.status = status_of(workspace);
   a.timeout_ns = g_timeout_ns;
 

@@ -410,18 +410,71 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           report_status(a.status, kStatusDeviceCheck, 0x5e1ec6u);
         const uint32_t b0 = sel.found_bin;
         const uint32_t need = (uint32_t)kk - sel.found_beyond;
-        const uint32_t cnt = hist[b0];
         named_bar_sync(bar_id, 128);   // hist of this token becomes scratch
+        // One pass over the candidates: entries above the cut-off bin are
+        // selected outright and written now; the cut-off bin's entries are
+        // gathered into this group's scratch, where the refinement runs.
+        const int64_t row = (int64_t)blk.b * a.nq + blk.t0 + st;
+        int32_t* idx_row = a.idx_out + row * a.k;
+        float* score_row = a.score_out ? a.score_out + row * a.k : nullptr;
+        uint2* bnd = a.bnd + ((int64_t)blockIdx.x * 4 + wg) * a.cand_cap;
+        if (tid == 0) {
+          sel.out_count = 0u;
+          sel.bnd_count = 0u;
+        }
+        named_bar_sync(bar_id, 128);
+        for (int j0 = 0; j0 < m; j0 += 128 * kBatch) {
+          uint32_t key[kBatch], pos[kBatch];
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u) {
+            key[u] = 0u;
+            pos[u] = 0u;
+            const int i = j0 + u * 128 + (int)tid;
+            if (i < m) get(i, key[u], pos[u]);
+          }
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u) {
+            const int i = j0 + u * 128 + (int)tid;
+            const uint32_t bin = score_bin(key[u]);
+            const bool above = i < m && bin > b0, on = i < m && bin == b0;
+            const uint32_t ma = __ballot_sync(0xffffffffu, above), mo = __ballot_sync(0xffffffffu, on);
+            uint32_t base_a = 0, base_o = 0;
+            if (lane == 0) {
+              if (ma) base_a = atomicAdd(&sel.out_count, (uint32_t)__popc(ma));
+              if (mo) base_o = atomicAdd(&sel.bnd_count, (uint32_t)__popc(mo));
+            }
+            base_a = __shfl_sync(0xffffffffu, base_a, 0);
+            base_o = __shfl_sync(0xffffffffu, base_o, 0);
+            const uint32_t below = (1u << lane) - 1u;
+            if (above) {
+              const uint32_t slot = base_a + __popc(ma & below);
+              if (slot < (uint32_t)kk) {
+                idx_row[slot] = (int32_t)pos[u];
+                if (score_row) score_row[slot] = key_to_float(key[u]);
+              }
+            }
+            if (on) {
+              const uint32_t slot = base_o + __popc(mo & below);
+              if (slot < (uint32_t)a.cand_cap) bnd[slot] = make_uint2(key[u], pos[u]);
+            }
+          }
+        }
+        named_bar_sync(bar_id, 128);
+        const int nb = (int)min((uint32_t)a.cand_cap, sel.bnd_count);
+        auto get_bnd = [bnd](int i, uint32_t& key, uint32_t& pos) {
+          const uint2 e = bnd[i];
+          key = e.x;
+          pos = e.y;
+        };
         SelectResult res;
         bin_key_range(b0, res.lo, res.hi);
         res.key_all_in = 1;
         res.pos_hi = 0;
-        if (need != cnt)
-          res = group_refine<128, kHistBins>(get, m, res.lo, res.hi, need, (uint32_t)tok_t[g], hist, sel, tid,
+        if (need != (uint32_t)nb)
+          res = group_refine<128, kHistBins>(get_bnd, nb, res.lo, res.hi, need, (uint32_t)tok_t[g], hist, sel, tid,
                                              bar_id, a.status);
-        const int64_t row = (int64_t)blk.b * a.nq + blk.t0 + st;
-        group_emit<128>(get, m, res, kk, a.k, a.idx_out + row * a.k,
-                        a.score_out ? a.score_out + row * a.k : nullptr, sel, tid, bar_id, a.status);
+        group_emit_append<128>(get_bnd, nb, res, kk, idx_row, score_row, sel, tid, bar_id);
+        group_emit_finish<128>(kk, a.k, idx_row, score_row, sel, tid, bar_id, a.status);
       }
     }
   }

@@ -38,6 +38,7 @@ struct PrefillArgs {
   float* score_out;            // [B, nq, k] or null
   uint2* cand;                 // [grid * 8, cand_cap] candidate (key, pos) buffers
   int64_t cand_cap;
+  uint2* bnd;                  // [grid * 4, cand_cap] cut-off bin entries of the row being selected
   DeviceStatus* status;
   uint64_t timeout_ns;
 };

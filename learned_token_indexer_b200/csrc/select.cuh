@@ -40,6 +40,7 @@ struct SelectShared {
   uint32_t found_beyond;
   uint32_t out_count;
   uint32_t aborted;
+  uint32_t bnd_count;
 };
 
 // Find the bin where the running count over `nbins` bins, traversed from the
@@ -235,6 +236,55 @@ __device__ void group_emit(Get get, int m, const SelectResult& r, int kk, int k,
   named_bar_sync(bar_id, NT);
   // A selection that does not produce exactly kk entries is a library bug:
   // report it and leave no stale slot behind.
+  const int got = (int)sh.out_count;
+  if (got != kk && tid == 0) report_status(status, kStatusDeviceCheck, 0x5e1ec7u);
+  for (int j = (got < kk ? got : kk) + (int)tid; j < k; j += NT) {
+    idx_row[j] = -1;
+    if (score_row) score_row[j] = -__int_as_float(0x7f800000);
+  }
+  named_bar_sync(bar_id, NT);
+}
+
+// Append the selected entries among entries [0, m) to idx_row / score_row at
+// slots counted on from sh.out_count (which the caller has set); no padding.
+template <int NT, typename Get>
+__device__ void group_emit_append(Get get, int m, const SelectResult& r, int kk, int32_t* idx_row, float* score_row,
+                                  SelectShared<NT>& sh, uint32_t tid, uint32_t bar_id) {
+  const uint32_t lane = tid & 31u;
+  for (int j0 = 0; j0 < m; j0 += NT * kBatch) {
+    uint32_t key[kBatch], pos[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      key[u] = 0u;
+      pos[u] = 0u;
+      const int i = j0 + u * NT + (int)tid;
+      if (i < m) get(i, key[u], pos[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = j0 + u * NT + (int)tid;
+      const bool sel = i < m && selected(r, key[u], pos[u]);
+      const uint32_t mask = __ballot_sync(0xffffffffu, sel);
+      uint32_t base = 0;
+      if (lane == 0 && mask) base = atomicAdd(&sh.out_count, (uint32_t)__popc(mask));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (sel) {
+        const uint32_t slot = base + __popc(mask & ((1u << lane) - 1u));
+        if (slot < (uint32_t)kk) {
+          idx_row[slot] = (int32_t)pos[u];
+          if (score_row) score_row[slot] = key_to_float(key[u]);
+        }
+      }
+    }
+  }
+  named_bar_sync(bar_id, NT);
+}
+
+// Check the emitted count (report a mismatch) and pad slots [count, k) with
+// -1 / -inf.
+template <int NT>
+__device__ void group_emit_finish(int kk, int k, int32_t* idx_row, float* score_row, SelectShared<NT>& sh,
+                                  uint32_t tid, uint32_t bar_id, DeviceStatus* status) {
   const int got = (int)sh.out_count;
   if (got != kk && tid == 0) report_status(status, kStatusDeviceCheck, 0x5e1ec7u);
   for (int j = (got < kk ? got : kk) + (int)tid; j < k; j += NT) {
