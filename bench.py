@@ -281,8 +281,10 @@ class DecodeRun:
         }
 
     def host_inputs(self):
-        return {k: v.cpu().pin_memory() for k, v in self.d.items()
-                if isinstance(v, torch.Tensor) and k != "lengths"}
+        """A decode step's host inputs: the new tokens' queries (q^I, w, q)
+        and the sequence offsets.  The K^I and latent caches are device state
+        that persists across steps, so they are not re-sent."""
+        return {k: self.d[k].cpu().pin_memory() for k in ("qI", "w", "q", "cu_seqlens")}
 
     def load_inputs(self, host):
         for k, v in host.items():
