@@ -32,28 +32,7 @@ namespace {
 constexpr int kQB = 8;          // tokens per block
 constexpr int kTA = 4;          // tokens per accumulator group
 constexpr int kPrefillThreads = 576;   // producer, MMA, 4 epilogue warpgroups
-constexpr int kHistBins = 512;  // streaming histogram bins (499 used)
-constexpr uint32_t kLastBin = 498;
-
-__device__ __forceinline__ uint32_t score_bin(uint32_t key) {
-  const uint32_t k11 = key >> 21;
-  if (k11 < 392u) return 0u;                    // x <= -2^31
-  if (k11 < 640u) return 1u + (k11 - 392u);     // -2^31 < x <= -2^-31
-  if (k11 < 1408u) return 249u;                 // |x| < 2^-31 (zeros)
-  if (k11 < 1656u) return 250u + (k11 - 1408u); // 2^-31 <= x < 2^31
-  return kLastBin;                              // x >= 2^31
-}
-
-__device__ __forceinline__ void bin_key_range(uint32_t b, uint32_t& lo, uint32_t& hi) {
-  uint32_t a, z;
-  if (b == 0u) { a = 0u; z = 391u; }
-  else if (b <= 248u) { a = z = 391u + b; }
-  else if (b == 249u) { a = 640u; z = 1407u; }
-  else if (b <= 497u) { a = z = 1408u + (b - 250u); }
-  else { a = 1656u; z = 2047u; }
-  lo = a << 21;
-  hi = (z << 21) | 0x1FFFFFu;
-}
+constexpr int kHistBins = kScoreBins;  // streaming histogram bins (499 used)
 
 // Raise a token's floor from its histogram (one warp): the bin where the
 // running count of accepted scores, from the top bin down, first reaches k
@@ -473,7 +452,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (need != (uint32_t)nb)
           res = group_refine<128, kHistBins>(get_bnd, nb, res.lo, res.hi, need, (uint32_t)tok_t[g], hist, sel, tid,
                                              bar_id, a.status);
-        group_emit_append<128>(get_bnd, nb, res, kk, idx_row, score_row, sel, tid, bar_id);
+        uint32_t blo, bhi;
+        bin_key_range(b0, blo, bhi);
+        group_emit_append<128>(get_bnd, nb, res, blo, bhi, kk, idx_row, score_row, sel, tid, bar_id);
         group_emit_finish<128>(kk, a.k, idx_row, score_row, sel, tid, bar_id, a.status);
       }
     }

@@ -26,6 +26,33 @@ namespace dsa {
 // loads in flight).
 constexpr int kBatch = 8;
 
+// Coarse monotone binning of score keys (the order-preserving uint32 image of
+// an fp32 score): quarter-octaves for 2^-31 <= |x| < 2^31, one bin for each
+// tail and one for |x| < 2^-31.  Larger key <=> same or higher bin.
+constexpr int kScoreBins = 512;      // bins 0..498 used
+constexpr uint32_t kScoreLastBin = 498;
+
+__device__ __forceinline__ uint32_t score_bin(uint32_t key) {
+  const uint32_t k11 = key >> 21;
+  if (k11 < 392u) return 0u;                    // x <= -2^31
+  if (k11 < 640u) return 1u + (k11 - 392u);     // -2^31 < x <= -2^-31
+  if (k11 < 1408u) return 249u;                 // |x| < 2^-31 (zeros)
+  if (k11 < 1656u) return 250u + (k11 - 1408u); // 2^-31 <= x < 2^31
+  return kScoreLastBin;                              // x >= 2^31
+}
+
+__device__ __forceinline__ void bin_key_range(uint32_t b, uint32_t& lo, uint32_t& hi) {
+  uint32_t a, z;
+  if (b == 0u) { a = 0u; z = 391u; }
+  else if (b <= 248u) { a = z = 391u + b; }
+  else if (b == 249u) { a = 640u; z = 1407u; }
+  else if (b <= 497u) { a = z = 1408u + (b - 250u); }
+  else { a = 1656u; z = 2047u; }
+  lo = a << 21;
+  hi = (z << 21) | 0x1FFFFFu;
+}
+
+
 struct SelectResult {
   uint32_t lo, hi;        // key interval of the cut-off
   uint32_t key_all_in;    // 1: every entry with key >= lo is selected
@@ -245,11 +272,13 @@ __device__ void group_emit(Get get, int m, const SelectResult& r, int kk, int k,
   named_bar_sync(bar_id, NT);
 }
 
-// Append the selected entries among entries [0, m) to idx_row / score_row at
-// slots counted on from sh.out_count (which the caller has set); no padding.
+// Append the selected entries with keys in [key_lo, key_hi] among entries
+// [0, m) to idx_row / score_row at slots counted on from sh.out_count (which
+// the caller has set); no padding.
 template <int NT, typename Get>
-__device__ void group_emit_append(Get get, int m, const SelectResult& r, int kk, int32_t* idx_row, float* score_row,
-                                  SelectShared<NT>& sh, uint32_t tid, uint32_t bar_id) {
+__device__ void group_emit_append(Get get, int m, const SelectResult& r, uint32_t key_lo, uint32_t key_hi, int kk,
+                                  int32_t* idx_row, float* score_row, SelectShared<NT>& sh, uint32_t tid,
+                                  uint32_t bar_id) {
   const uint32_t lane = tid & 31u;
   for (int j0 = 0; j0 < m; j0 += NT * kBatch) {
     uint32_t key[kBatch], pos[kBatch];
@@ -263,7 +292,7 @@ __device__ void group_emit_append(Get get, int m, const SelectResult& r, int kk,
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int i = j0 + u * NT + (int)tid;
-      const bool sel = i < m && selected(r, key[u], pos[u]);
+      const bool sel = i < m && key[u] >= key_lo && key[u] <= key_hi && selected(r, key[u], pos[u]);
       const uint32_t mask = __ballot_sync(0xffffffffu, sel);
       uint32_t base = 0;
       if (lane == 0 && mask) base = atomicAdd(&sh.out_count, (uint32_t)__popc(mask));

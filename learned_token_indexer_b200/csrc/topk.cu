@@ -3,11 +3,13 @@
 // separate radix top-k that handles variable-length rows via seq_lens), plus
 // small helper kernels.
 //
-// One CTA (1024 threads) per row; 2048-bin digit histograms in shared memory.
-// The first refinement pass histograms the top 11 bits of every score's
-// order-preserving key; later passes only count entries still inside the
-// cut-off interval.  Used by the decode step (64 rows of 4096..65536 scores)
-// and by the debug path.
+// One CTA (1024 threads) per row, two passes over the row in the usual case:
+// a histogram of the row's scores over the coarse score bins finds the
+// cut-off bin; one pass then writes every entry above that bin and gathers
+// the cut-off bin's entries into shared memory, where the exact radix
+// refinement on (key, position) runs.  (A cut-off bin too large for shared
+// memory is refined over the row instead.)  Used by the decode step (64 rows
+// of 4096..65536 scores) and by the debug path.
 #include "kernels.h"
 #include "select.cuh"
 
@@ -15,14 +17,16 @@ namespace dsa {
 
 namespace {
 constexpr int kRowThreads = 1024;
-constexpr int kRowBins = 2048;
+constexpr int kRowBins = 2048;        // refinement digit bins
+constexpr int kBndCap = 4096;         // cut-off bin entries kept in shared memory
 }  // namespace
 
 __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRowsArgs a) {
   __shared__ uint32_t hist[kRowBins];
+  __shared__ uint2 bnd[kBndCap];
   __shared__ SelectShared<kRowThreads> sh;
   const int row = blockIdx.x;
-  const uint32_t tid = threadIdx.x;
+  const uint32_t tid = threadIdx.x, lane = tid & 31u;
   const float* src;
   int len;
   if (a.cu_seqlens) {
@@ -45,17 +49,105 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRow
     key = float_to_key(src[i]);
     pos = (uint32_t)i;
   };
+  if (kk == 0 || kk == len) {
+    // nothing to choose: every entry (or none) is selected
+    SelectResult r;
+    r.lo = kk > 0 ? 0u : 0xFFFFFFFFu;
+    r.hi = 0xFFFFFFFFu;
+    r.key_all_in = 1;
+    r.pos_hi = 0;
+    group_emit<kRowThreads>(get, kk > 0 ? len : 0, r, kk, a.k, idx_row, val_row, sh, tid, 0, a.status);
+    return;
+  }
+  // ---- pass 1: coarse score-bin histogram of the row
+  for (int i = (int)tid; i < kScoreBins; i += kRowThreads) hist[i] = 0u;
+  __syncthreads();
+  for (int j0 = 0; j0 < len; j0 += kRowThreads * kBatch) {
+    uint32_t key[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = j0 + u * kRowThreads + (int)tid;
+      key[u] = i < len ? float_to_key(src[i]) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = j0 + u * kRowThreads + (int)tid;
+      if (i < len) atomicAdd(&hist[score_bin(key[u])], 1u);
+    }
+  }
+  __syncthreads();
+  if (!group_find<kRowThreads>(hist, kScoreBins, (uint32_t)kk, true, sh, tid, 0) && tid == 0)
+    report_status(a.status, kStatusDeviceCheck, 0x5e1ec5u);
+  const uint32_t b0 = sh.found_bin;
+  const uint32_t need = (uint32_t)kk - sh.found_beyond;
+  uint32_t blo, bhi;
+  bin_key_range(b0, blo, bhi);
+  // ---- pass 2: entries above the cut-off bin are selected outright; the
+  // cut-off bin's entries go to shared memory
+  if (tid == 0) {
+    sh.out_count = 0u;
+    sh.bnd_count = 0u;
+  }
+  __syncthreads();
+  for (int j0 = 0; j0 < len; j0 += kRowThreads * kBatch) {
+    uint32_t key[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = j0 + u * kRowThreads + (int)tid;
+      key[u] = i < len ? float_to_key(src[i]) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = j0 + u * kRowThreads + (int)tid;
+      const bool above = i < len && key[u] > bhi, on = i < len && key[u] >= blo && key[u] <= bhi;
+      const uint32_t ma = __ballot_sync(0xffffffffu, above), mo = __ballot_sync(0xffffffffu, on);
+      uint32_t base_a = 0, base_o = 0;
+      if (lane == 0) {
+        if (ma) base_a = atomicAdd(&sh.out_count, (uint32_t)__popc(ma));
+        if (mo) base_o = atomicAdd(&sh.bnd_count, (uint32_t)__popc(mo));
+      }
+      base_a = __shfl_sync(0xffffffffu, base_a, 0);
+      base_o = __shfl_sync(0xffffffffu, base_o, 0);
+      const uint32_t below = (1u << lane) - 1u;
+      if (above) {
+        const uint32_t slot = base_a + __popc(ma & below);
+        if (slot < (uint32_t)kk) {
+          idx_row[slot] = i;
+          if (val_row) val_row[slot] = key_to_float(key[u]);
+        }
+      }
+      if (on) {
+        const uint32_t slot = base_o + __popc(mo & below);
+        if (slot < (uint32_t)kBndCap) bnd[slot] = make_uint2(key[u], (uint32_t)i);
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t nb = sh.bnd_count;
   SelectResult r;
-  r.lo = 0xFFFFFFFFu;
-  r.hi = 0xFFFFFFFFu;
+  r.lo = blo;
+  r.hi = bhi;
   r.key_all_in = 1;
   r.pos_hi = 0;
-  if (kk > 0 && kk < len)
-    r = group_refine<kRowThreads, kRowBins>(get, len, 0u, 0xFFFFFFFFu, (uint32_t)kk, (uint32_t)(len - 1), hist, sh,
-                                             tid, 0, a.status);
-  else if (kk == len && len > 0)
-    r.lo = 0u;   // every entry is selected
-  group_emit<kRowThreads>(get, kk > 0 ? len : 0, r, kk, a.k, idx_row, val_row, sh, tid, 0, a.status);
+  if (nb <= (uint32_t)kBndCap) {
+    auto get_bnd = [](int i, uint32_t& key, uint32_t& pos) {
+      const uint2 e = bnd[i];
+      key = e.x;
+      pos = e.y;
+    };
+    if (need != nb)
+      r = group_refine<kRowThreads, kRowBins>(get_bnd, (int)nb, blo, bhi, need, (uint32_t)(len - 1), hist, sh, tid,
+                                              0, a.status);
+    group_emit_append<kRowThreads>(get_bnd, (int)nb, r, blo, bhi, kk, idx_row, val_row, sh, tid, 0);
+  } else {
+    // the cut-off bin does not fit: refine and emit over the row, taking only
+    // entries inside the bin (those above it are already written)
+    if (need != nb)
+      r = group_refine<kRowThreads, kRowBins>(get, len, blo, bhi, need, (uint32_t)(len - 1), hist, sh, tid, 0,
+                                              a.status);
+    group_emit_append<kRowThreads>(get, len, r, blo, bhi, kk, idx_row, val_row, sh, tid, 0);
+  }
+  group_emit_finish<kRowThreads>(kk, a.k, idx_row, val_row, sh, tid, 0, a.status);
 }
 
 cudaError_t launch_topk_rows(const TopkRowsArgs& a, cudaStream_t stream) {
