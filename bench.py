@@ -256,7 +256,8 @@ class DecodeRun:
         if ev is not None:
             ev["idx"][0].append(PrefillRun._rec())
         dsa.indexer_topk_decode(d["qI"], d["w"], d["kI_cache"], d["cu_seqlens"], w.k, self.total, self.maxlen,
-                                idx_out=self.idx, workspace=self.ws_idx)
+                                q_scale=d.get("q_scale"), k_scale=d.get("k_scale"), idx_out=self.idx,
+                                workspace=self.ws_idx)
         if ev is not None:
             ev["idx"][1].append(PrefillRun._rec())
         dsa.sparse_attn_decode(d["q"], d["latent_cache"], d["cu_seqlens"], self.idx, w.Dv, self.total,
@@ -269,11 +270,13 @@ class DecodeRun:
 
     def kernel_work(self):
         w = self.w
-        scan_bytes = self.total * w.dI * 2 + w.B * w.HI * (w.dI * 2 + 4) + self.total * 4 * 2
+        eb = 1 if w.fp8 else 2   # K^I bytes per element (FP8 adds one fp32 scale per key)
+        scan_bytes = self.total * (w.dI * eb + (4 if w.fp8 else 0)) + w.B * w.HI * (w.dI * eb + 4) + self.total * 4 * 2
         gather = w.B * w.k * w.Dqk * 2
         return {
             "indexer_topk_decode": {"bytes": scan_bytes, "unit": "GB/s",
-                                    "per_unit": f"dI*2 = {w.dI * 2} B of K^I per cached key (+ q, w, fp32 scores)",
+                                    "per_unit": (f"dI*{eb} = {w.dI * eb} B of K^I per cached key"
+                                                 f"{' + 4 B scale' if w.fp8 else ''} (+ q, w, fp32 scores)"),
                                     "units": self.total},
             "sparse_attn_decode": {"bytes": gather + w.B * w.H * (w.Dqk + w.Dv) * 2, "unit": "GB/s",
                                    "per_unit": f"Dqk*2 = {w.Dqk * 2} B per selected latent row (+ q, out)",
@@ -284,7 +287,8 @@ class DecodeRun:
         """A decode step's host inputs: the new tokens' queries (q^I, w, q)
         and the sequence offsets.  The K^I and latent caches are device state
         that persists across steps, so they are not re-sent."""
-        return {k: self.d[k].cpu().pin_memory() for k in ("qI", "w", "q", "cu_seqlens")}
+        keys = ("qI", "w", "q", "cu_seqlens") + (("q_scale",) if "q_scale" in self.d else ())
+        return {k: self.d[k].cpu().pin_memory() for k in keys}
 
     def load_inputs(self, host):
         for k, v in host.items():
@@ -340,14 +344,13 @@ def cpu_baseline(w: W.Workload, budget_s: float = 15.0, run_inputs=None):
     if w.kind == "decode":
         d = run_inputs if run_inputs is not None else W.make_decode_inputs(w, "cpu")
         cu = d["cu_seqlens"].cpu().numpy()
-        q = d["qI"].cpu().double().numpy()
         ww = d["w"].cpu().double().numpy()
         t0 = time.perf_counter()
         done = 0
         for b in range(w.B):
             lo, hi = int(cu[b]), int(cu[b + 1])
-            kc = d["kI_cache"][lo:hi].cpu().double().numpy()
-            s = O.indexer_scores_row(q[b], kc, ww[b])
+            qb, kc = _decode_indexer_host(O, w, d, b, lo, hi)
+            s = O.indexer_scores_row(qb, kc, ww[b])
             sel = O.causal_topk_row(s, hi - lo - 1, w.k)
             lat = d["latent_cache"][lo:hi].cpu().double().numpy()
             O.sparse_attention_row(d["q"][b].cpu().double().numpy(), lat, sel, w.scale, w.Dv)
@@ -387,6 +390,15 @@ def _oracle_row(O, w, d, b, i):
     O.sparse_attention_row(d["q"][b, i].double().numpy(), lat, sel, w.scale, w.Dv)
 
 
+def _decode_indexer_host(O, w, d, b, lo, hi):
+    """Float64 q^I of sequence b and its K^I cache rows (dequantised for FP8)."""
+    if w.fp8:
+        q = O.dequantize(d["qI"][b].view(torch.uint8).cpu().numpy(), d["q_scale"][b].cpu().numpy(), 2)
+        k = O.dequantize(d["kI_cache"][lo:hi].view(torch.uint8).cpu().numpy(), d["k_scale"][lo:hi].cpu().numpy(), 1)
+        return q, k
+    return d["qI"][b].cpu().double().numpy(), d["kI_cache"][lo:hi].cpu().double().numpy()
+
+
 def _blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -400,7 +412,8 @@ def _blas_threads():
 
 def workload_label(w: W.Workload):
     if w.kind == "decode":
-        return (f"decode B={w.B} L~U[{w.L_min},{w.L_max}] HI={w.HI} dI={w.dI} k={w.k} bf16 K^I cache; "
+        return (f"decode B={w.B} L~U[{w.L_min},{w.L_max}] HI={w.HI} dI={w.dI} k={w.k} "
+                f"{'fp8-e4m3' if w.fp8 else 'bf16'} K^I cache; "
                 f"attn H={w.H} latent {w.Dqk}/{w.Dv}")
     dt = "fp8-e4m3 indexer" if w.fp8 else ("bf16 integer-valued indexer" if w.integer_valued else "bf16 indexer")
     ch = f" in {w.chunk}-query chunks" if w.chunk else ""
@@ -546,8 +559,8 @@ def run_reference(args):
         cu = d["cu_seqlens"].numpy()
         def one(b):
             lo, hi = int(cu[b]), int(cu[b + 1])
-            s = O.indexer_scores_row(d["qI"][b].double().numpy(), d["kI_cache"][lo:hi].double().numpy(),
-                                     d["w"][b].double().numpy())
+            qb, kc = _decode_indexer_host(O, w, d, b, lo, hi)
+            s = O.indexer_scores_row(qb, kc, d["w"][b].double().numpy())
             sel = O.causal_topk_row(s, hi - lo - 1, w.k)
             O.sparse_attention_row(d["q"][b].double().numpy(), d["latent_cache"][lo:hi].double().numpy(), sel,
                                    w.scale, w.Dv)

@@ -63,10 +63,12 @@ PREFILL_FP8 = Workload("prefill_fp8", "prefill", B=2, n=32768, HI=64, dI=128, k=
                        Dqk=576, Dv=512, qk_dist="normal", w_std=0.1, fp8=True, seed=2)
 DECODE = Workload("decode", "decode", B=64, n=0, HI=64, dI=128, k=2048, H=128, Dqk=576, Dv=512,
                   qk_dist="normal", w_std=0.1, seed=3, L_min=4096, L_max=65536)
+DECODE_FP8 = Workload("decode_fp8", "decode", B=64, n=0, HI=64, dI=128, k=2048, H=128, Dqk=576, Dv=512,
+                      qk_dist="normal", w_std=0.1, fp8=True, seed=3, L_min=4096, L_max=65536)
 LONG = Workload("long_prefill", "prefill", B=1, n=131072, HI=64, dI=128, k=2048, H=16, Dqk=576,
                 Dv=512, qk_dist="normal", w_std=0.1, chunk=8192, seed=4)
 
-ALL = {w.name: w for w in (TINY, PREFILL, PREFILL_FP8, DECODE, LONG)}
+ALL = {w.name: w for w in (TINY, PREFILL, PREFILL_FP8, DECODE, DECODE_FP8, LONG)}
 
 
 def scaled(w: Workload, **changes) -> Workload:
@@ -142,6 +144,8 @@ def make_decode_inputs(w: Workload, device="cpu", lengths: Optional[torch.Tensor
     Returns cu_seqlens int64 [B+1] (device), lengths (CPU),
       qI [B,HI,dI] bf16, w [B,HI] fp32, kI_cache [sum L, dI] bf16,
       q [B,H,Dqk] bf16, latent_cache [sum L, Dqk] bf16.
+    FP8 workloads draw the same bf16 values, then quantise q^I per query
+    token (q_scale [B]) and the K^I cache per key (k_scale [sum L]) to e4m3.
     """
     lengths = decode_lengths(w) if lengths is None else lengths
     B = lengths.numel()
@@ -155,6 +159,9 @@ def make_decode_inputs(w: Workload, device="cpu", lengths: Optional[torch.Tensor
     out["kI_cache"] = torch.randn((total, w.dI), generator=g, device=device).to(torch.bfloat16)
     out["q"] = torch.randn((B, w.H, w.Dqk), generator=g, device=device).to(torch.bfloat16)
     out["latent_cache"] = torch.randn((total, w.Dqk), generator=g, device=device).to(torch.bfloat16)
+    if w.fp8:
+        out["qI"], out["q_scale"] = quantize_fp8_per_token(out["qI"], 2)
+        out["kI_cache"], out["k_scale"] = quantize_fp8_per_token(out["kI_cache"], 1)
     return out
 
 

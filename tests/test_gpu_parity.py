@@ -18,7 +18,7 @@ import learned_token_indexer_b200 as dsa
 import oracle as O
 from learned_token_indexer_b200 import workloads as W
 from tests import checks
-from tests.gpu_util import host_f64, indexer_host_inputs
+from tests.gpu_util import host_dequant, host_f64, indexer_host_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -322,17 +322,22 @@ def test_worked_example_through_the_library():
 # decode
 # --------------------------------------------------------------------------
 
-def _decode_case(w, lengths, fp8=False):
+def _decode_case(w, lengths):
     d = W.make_decode_inputs(w, "cuda", lengths=lengths)
     total, maxlen = int(lengths.sum()), int(lengths.max())
     ws = _ws()
-    idx = dsa.indexer_topk_decode(d["qI"], d["w"], d["kI_cache"], d["cu_seqlens"], w.k, total, maxlen, workspace=ws)
+    idx = dsa.indexer_topk_decode(d["qI"], d["w"], d["kI_cache"], d["cu_seqlens"], w.k, total, maxlen,
+                                  q_scale=d.get("q_scale"), k_scale=d.get("k_scale"), workspace=ws)
     out, lse = dsa.sparse_attn_decode(d["q"], d["latent_cache"], d["cu_seqlens"], idx, w.Dv, total, scale=w.scale,
                                       return_lse=True, workspace=ws)
     torch.cuda.synchronize()
     _no_device_errors(ws)
     cu = d["cu_seqlens"].cpu().numpy()
-    qh, kh, wh = host_f64(d["qI"]), host_f64(d["kI_cache"]), host_f64(d["w"])
+    if w.fp8:   # the oracle scores the dequantised codes (the quantisation is an input)
+        qh, kh = host_dequant(d["qI"], d["q_scale"], 2), host_dequant(d["kI_cache"], d["k_scale"], 1)
+    else:
+        qh, kh = host_f64(d["qI"]), host_f64(d["kI_cache"])
+    wh = host_f64(d["w"])
     idx_h = idx.cpu().numpy()
     bad = []
     for b in range(len(lengths)):
@@ -351,9 +356,20 @@ def test_decode_small_ragged():
     _decode_case(w, torch.tensor([1, 129, 300, 1000, 4097]))
 
 
+def test_decode_fp8_cache_small_ragged():
+    # e4m3 K^I cache with one scale per key, e4m3 queries with one scale per token
+    w = W.scaled(W.DECODE_FP8, B=5, k=300)
+    _decode_case(w, torch.tensor([1, 129, 300, 1000, 4097]))
+
+
 @pytest.mark.slow
 def test_decode_full_workload():
     _decode_case(W.DECODE, W.decode_lengths(W.DECODE))
+
+
+@pytest.mark.slow
+def test_decode_fp8_full_workload():
+    _decode_case(W.DECODE_FP8, W.decode_lengths(W.DECODE_FP8))
 
 
 # --------------------------------------------------------------------------
