@@ -76,13 +76,25 @@ __device__ __forceinline__ void raise_floor(const uint32_t* hist, uint32_t k, ui
   }
 }
 
+// Accumulator plan: each TMEM accumulator holds the heads of kTPA tokens of
+// the block (MMA N = kTPA * HI).  Two tokens per accumulator (four
+// accumulators, one per epilogue warpgroup, which releases it alone) where the
+// MMA shape allows it (N >= 16); four tokens otherwise (two accumulators,
+// every warpgroup reading one token of each).
+template <int HI>
+struct AccPlan {
+  static constexpr int kTPA = (2 * HI >= 16) ? 2 : 4;
+  static constexpr int kNA = kQB / kTPA;
+  static constexpr int kNP = kTPA * HI;
+};
+
 struct Block {
   int b, t0;      // sequence, first local query row
   int nvalid;     // valid tokens in the block (<= 8)
-  int nt[2];      // key tiles per group (0 = group empty)
+  int nt[4];      // key tiles per accumulator (0 = no valid token in it)
 };
 
-__device__ __forceinline__ bool block_of(const PrefillArgs& a, int r, Block& blk) {
+__device__ __forceinline__ bool block_of(const PrefillArgs& a, int r, Block& blk, int tpa) {
   // Round r of the snake schedule: CTA c takes item r*G + (c or G-1-c).
   const int G = gridDim.x;
   const int c = blockIdx.x;
@@ -94,15 +106,16 @@ __device__ __forceinline__ bool block_of(const PrefillArgs& a, int r, Block& blk
   const int bi = a.nblk - 1 - j;   // heaviest (last) blocks first
   blk.t0 = bi * kQB;
   blk.nvalid = min(kQB, a.nq - blk.t0);
-  for (int g = 0; g < 2; ++g) {
-    const int last = min(blk.t0 + kTA * g + kTA - 1, a.nq - 1);
-    if (blk.t0 + kTA * g >= a.nq) {
+  for (int g = 0; g < kQB / tpa; ++g) {
+    const int last = min(blk.t0 + tpa * g + tpa - 1, a.nq - 1);
+    if (blk.t0 + tpa * g >= a.nq) {
       blk.nt[g] = 0;
     } else {
       const int tmax = a.q_offset + last;
       blk.nt[g] = tmax / kTileKeys + 1;
     }
   }
+  for (int g = kQB / tpa; g < 4; ++g) blk.nt[g] = 0;
   return true;
 }
 
@@ -112,11 +125,13 @@ template <int HI, bool FP8, int KB, int STAGES>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     indexer_topk_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,
                                 const __grid_constant__ CUtensorMap tmap_k, const PrefillArgs a) {
-  constexpr int N = kTA * HI;                                 // MMA N per group
+  constexpr int N = kTA * HI;                                 // Q rows per TMA group (4 tokens)
+  using Plan = AccPlan<HI>;
+  constexpr int kNA = Plan::kNA, kNP = Plan::kNP, kTPA = Plan::kTPA;
   constexpr int kQGroupBytes = N * KB * kSwizzleBytes;
   constexpr int kKBytes = kTileKeys * KB * kSwizzleBytes;
   constexpr uint32_t kTmemCols = (2 * N <= 32) ? 32 : (2 * N <= 64 ? 64 : (2 * N <= 128 ? 128 : (2 * N <= 256 ? 256 : 512)));
-  constexpr uint32_t kIdesc = instr_desc(ElemTraits<FP8>::kFormat, kTileKeys, N);
+  constexpr uint32_t kIdesc = instr_desc(ElemTraits<FP8>::kFormat, kTileKeys, kNP);
   constexpr int kElemsPerBlock = ElemTraits<FP8>::kElemsPerBlock;
 
   extern __shared__ uint8_t smem_raw[];
@@ -134,9 +149,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   uint64_t* k_empty = bars + STAGES;
   uint64_t* q_full = bars + 2 * STAGES;
   uint64_t* q_empty = q_full + 1;
-  uint64_t* acc_full = q_empty + 1;   // [2]
-  uint64_t* acc_empty = acc_full + 2; // [2]
-  uint64_t* mma_done = acc_empty + 2;
+  uint64_t* acc_full = q_empty + 1;   // [kNA]
+  uint64_t* acc_empty = acc_full + 4; // [kNA]
+  uint64_t* mma_done = acc_empty + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
 
@@ -148,9 +163,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    for (int g = 0; g < 2; ++g) {
+    for (int g = 0; g < kNA; ++g) {
       mbar_init(&acc_full[g], 1);
-      mbar_init(&acc_empty[g], 16);
+      mbar_init(&acc_empty[g], kNA == 4 ? 4 : 16);   // the owning warpgroup, or all four
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0u;
@@ -182,7 +197,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       uint32_t q_last_parity = 0;
       bool ok = true;
       Block blk;
-      for (int r = 0; ok && block_of(a, r, blk); ++r) {
+      for (int r = 0; ok && block_of(a, r, blk, kTPA); ++r) {
         if (!(ok = mbar_wait(q_empty, qphase ^ 1u, ctl, 0x1101))) break;
         mbar_arrive_expect_tx(q_full, 2 * kQGroupBytes);
         for (int g = 0; g < 2; ++g)
@@ -192,7 +207,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         q_issued = true;
         q_last_parity = qphase;
         qphase ^= 1u;
-        const int nt = max(blk.nt[0], blk.nt[1]);
+        const int nt = max(max(blk.nt[0], blk.nt[1]), max(blk.nt[2], blk.nt[3]));
         for (int t = 0; t < nt; ++t) {
           if (!(ok = mbar_wait(&k_empty[stage], kphase ^ 1u, ctl, 0x1102))) break;
           mbar_arrive_expect_tx(&k_full[stage], kKBytes);
@@ -223,24 +238,28 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
       int stage = 0;
-      uint32_t kphase = 0, qphase = 0, aphase[2] = {0u, 0u};
+      uint32_t kphase = 0, qphase = 0, aphase[4] = {0u, 0u, 0u, 0u};
       bool ok = true;
       Block blk;
-      for (int r = 0; ok && block_of(a, r, blk); ++r) {
+      for (int r = 0; ok && block_of(a, r, blk, kTPA); ++r) {
         if (!(ok = mbar_wait(q_full, qphase, ctl, 0x1201))) break;
         qphase ^= 1u;
         tc_fence_after();
-        const int nt = max(blk.nt[0], blk.nt[1]);
+        const int nt = max(max(blk.nt[0], blk.nt[1]), max(blk.nt[2], blk.nt[3]));
         for (int t = 0; t < nt && ok; ++t) {
           if (!(ok = mbar_wait(&k_full[stage], kphase, ctl, 0x1202))) break;
           tc_fence_after();
-          for (int g = 0; g < 2; ++g) {
+#pragma unroll
+          for (int g = 0; g < kNA; ++g) {
             if (t >= blk.nt[g]) continue;
             if (!(ok = mbar_wait(&acc_empty[g], aphase[g] ^ 1u, ctl, 0x1203))) break;
             aphase[g] ^= 1u;
             tc_fence_after();
-            issue_tile_mma<FP8>(tmem_base + g * N, smem_u32(sK + stage * kKBytes), smem_u32(sQ + g * kQGroupBytes),
-                                N, a.ksteps, kIdesc);
+            // accumulator g holds Q rows [g*kNP, (g+1)*kNP): inside TMA group
+            // (g*kTPA)/4 at row (g*kTPA)%4 * HI; K blocks are N rows apart
+            const int grp = (g * kTPA) / kTA, row0 = ((g * kTPA) % kTA) * HI;
+            issue_tile_mma<FP8>(tmem_base + g * kNP, smem_u32(sK + stage * kKBytes),
+                                smem_u32(sQ + grp * kQGroupBytes + row0 * kSwizzleBytes), N, a.ksteps, kIdesc);
             tc_commit(&acc_full[g]);
           }
           if (!ok) break;
@@ -258,11 +277,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
-    // Four warpgroups; warpgroup j owns block token j of accumulator group 0
-    // and token 4+j of group 1 (columns [j*HI, (j+1)*HI) of each group).
-    // Every thread of a warpgroup runs the same sequence of named barriers; a
-    // wait that fails only turns the remaining work into no-ops (no early
-    // exit, so no barrier is ever left short of threads).
+    // Four warpgroups, two block tokens each (token u of warpgroup j is block
+    // slot st = ST(j, u)): with four accumulators warpgroup j owns accumulator
+    // j (tokens 2j, 2j+1); with two, it takes token j of accumulator 0 and
+    // token 4+j of accumulator 1.  Every thread of a warpgroup runs the same
+    // sequence of named barriers; a wait that fails only turns the remaining
+    // work into no-ops (no early exit, so no barrier is left short of threads).
     const uint32_t wg = (warp - 2) >> 2;                  // 0..3
     const uint32_t tid = (warp - 2 - 4 * wg) * 32 + lane; // 0..127 inside the warpgroup
     const uint32_t bar_id = 2 + wg;
@@ -270,93 +290,116 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint32_t lane_grp = quarter * 32u;
     const uint32_t key_in_tile = lane_grp + lane;
     SelectShared<128>& sel = sSel[wg];
+    // block slot, accumulator and accumulator column of token u of this group
+    auto ST = [&](int u) { return kNA == 4 ? 2 * (int)wg + u : kTA * u + (int)wg; };
+    auto ACC = [&](int u) { return kNA == 4 ? (int)wg : u; };
     uint32_t aphase[2] = {0u, 0u};
     bool ok = true;
     Block blk;
-    for (int r = 0; block_of(a, r, blk); ++r) {
+    for (int r = 0; block_of(a, r, blk, kTPA); ++r) {
       named_bar_sync(bar_id, 128);
-      // per-block state of this warpgroup's 2 tokens (slot st = 4*g + wg)
       int tok_t[2];
       bool tok_valid[2];
+      int tok_nt[2];   // key tiles of the accumulator holding token u
 #pragma unroll
-      for (int g = 0; g < 2; ++g) {
-        const int li = blk.t0 + kTA * g + (int)wg;
-        tok_valid[g] = li < a.nq;
-        tok_t[g] = a.q_offset + li;
+      for (int u = 0; u < 2; ++u) {
+        const int li = blk.t0 + ST(u);
+        tok_valid[u] = li < a.nq;
+        tok_t[u] = a.q_offset + li;
+        tok_nt[u] = blk.nt[ACC(u)];
       }
       for (int i = (int)tid; i < 2 * kHistBins; i += 128) {
-        const int g = i / kHistBins;
-        sHist[(kTA * g + wg) * kHistBins + (i - g * kHistBins)] = 0u;
+        const int u = i / kHistBins;
+        sHist[ST(u) * kHistBins + (i - u * kHistBins)] = 0u;
       }
-      if (tid < 2u) sFloorKey[kTA * tid + wg] = 0u;   // key 0: every score passes
+      if (tid < 2u) sFloorKey[ST((int)tid)] = 0u;   // key 0: every score passes
       for (int i = (int)tid; i < 2 * HI; i += 128) {
-        const int g = i / HI, h = i - g * HI;
-        const int li = blk.t0 + kTA * g + (int)wg;
+        const int u = i / HI, h = i - u * HI;
+        const int li = blk.t0 + ST(u);
         float wv = 0.0f;
         if (li < a.nq) {
           const int64_t row = (int64_t)blk.b * a.nq + li;
           wv = a.w[row * HI + h];
           if (FP8) wv *= a.q_scale[row];
         }
-        sW[(kTA * g + wg) * HI + h] = wv;
+        sW[ST(u) * HI + h] = wv;
       }
       named_bar_sync(bar_id, 128);
-      const int nt_max = max(blk.nt[0], blk.nt[1]);
+      const int nt_max = max(tok_nt[0], tok_nt[1]);
       // accepted (key, position) pairs: this warp's sub-buffer of each token
       // (warp q of the group sees keys with s mod 128 in [32q, 32q + 32))
       uint2* cand_w[2];
       uint32_t cnt[2] = {0u, 0u};
 #pragma unroll
-      for (int g = 0; g < 2; ++g)
-        cand_w[g] = a.cand + ((int64_t)blockIdx.x * kQB + kTA * g + wg) * a.cand_cap + quarter * (a.cand_cap / 4);
+      for (int u = 0; u < 2; ++u)
+        cand_w[u] = a.cand + ((int64_t)blockIdx.x * kQB + ST(u)) * a.cand_cap + quarter * (a.cand_cap / 4);
       for (int t = 0; t < nt_max; ++t) {
         const int s = t * kTileKeys + (int)key_in_tile;
         float ks = 1.0f;
         if (FP8 && ok) ks = (s < a.kv_len) ? a.k_scale[(int64_t)blk.b * a.kv_len + s] : 0.0f;
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          if (t >= blk.nt[g]) continue;
-          const bool got = ok && mbar_wait(&acc_full[g], aphase[g], ctl, 0x1301);
+        float score[2] = {0.0f, 0.0f};
+        if constexpr (kNA == 4) {
+          // both tokens in this group's own accumulator: one wait, one release
+          const bool got = ok && mbar_wait(&acc_full[wg], aphase[0], ctl, 0x1301);
           ok = __all_sync(0xffffffffu, got);
-          aphase[g] ^= 1u;
-          if (!ok) continue;
-          tc_fence_after();
-          float sc[1];
-          group_head_sums<HI, 1>(tmem_base + (lane_grp << 16) + g * N + wg * HI, sW + (kTA * g + wg) * HI, sc,
-                                 &acc_empty[g], lane);
-          const float score = FP8 ? sc[0] * ks : sc[0];
+          aphase[0] ^= 1u;
+          if (ok) {
+            tc_fence_after();
+            group_head_sums<HI, 2>(tmem_base + (lane_grp << 16) + wg * kNP, sW + ST(0) * HI, score, &acc_empty[wg],
+                                   lane);
+          }
+        } else {
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            if (t >= tok_nt[u]) continue;
+            const bool got = ok && mbar_wait(&acc_full[u], aphase[u], ctl, 0x1301);
+            ok = __all_sync(0xffffffffu, got);
+            aphase[u] ^= 1u;
+            if (!ok) continue;
+            tc_fence_after();
+            float sc[1];
+            group_head_sums<HI, 1>(tmem_base + (lane_grp << 16) + u * kNP + wg * HI, sW + ST(u) * HI, sc,
+                                   &acc_empty[u], lane);
+            score[u] = sc[0];
+          }
+        }
+        if (!ok) continue;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (t >= tok_nt[u]) continue;
+          const float sc_u = FP8 ? score[u] * ks : score[u];
           // streaming filter: a key below the token's floor cannot be in its
           // top k (the floor only rises; another warp may raise it meanwhile)
-          const int st = kTA * g + (int)wg;
-          const uint32_t key = float_to_key(score);
+          const int st = ST(u);
+          const uint32_t key = float_to_key(sc_u);
           const uint32_t floor_key = *reinterpret_cast<volatile const uint32_t*>(&sFloorKey[st]);
-          const bool acc = tok_valid[g] && s <= tok_t[g] && key >= floor_key;
+          const bool acc = tok_valid[u] && s <= tok_t[u] && key >= floor_key;
           const uint32_t mask = __ballot_sync(0xffffffffu, acc);
           if (acc) {
-            cand_w[g][cnt[g] + __popc(mask & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)s);
+            cand_w[u][cnt[u] + __popc(mask & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)s);
             // histogram of accepted scores, one atomic per distinct bin of the warp
             const uint32_t bin = score_bin(key);
             const uint32_t peers = __match_any_sync(mask, bin);
             if (lane == (uint32_t)(__ffs(peers) - 1)) atomicAdd(&sHist[st * kHistBins + bin], (uint32_t)__popc(peers));
           }
-          cnt[g] += (uint32_t)__popc(mask);
-          // raise the floor (warp q = g of the group, every tile): the bin
+          cnt[u] += (uint32_t)__popc(mask);
+          // raise the floor (warp q = u of the group, every tile): the bin
           // where the count of accepted scores from the top first reaches k
-          if (quarter == (uint32_t)g) raise_floor(sHist + st * kHistBins, (uint32_t)a.k, &sFloorKey[st], lane);
+          if (quarter == (uint32_t)u) raise_floor(sHist + st * kHistBins, (uint32_t)a.k, &sFloorKey[st], lane);
         }
       }
       // per-warp candidate counts for the select
 #pragma unroll
-      for (int g = 0; g < 2; ++g)
-        if (lane == 0) sCnt[(kTA * g + wg) * 4 + quarter] = cnt[g];
+      for (int u = 0; u < 2; ++u)
+        if (lane == 0) sCnt[ST(u) * 4 + quarter] = cnt[u];
       named_bar_sync(bar_id, 128);
       if (tid == 0) sel.aborted = *abort_flag;
       named_bar_sync(bar_id, 128);
       if (sel.aborted) continue;   // warpgroup-uniform: nothing below is valid
       // ---- exact select of each token's top min(k, t+1)
       for (int g = 0; g < 2; ++g) {
-        if (!tok_valid[g] || blk.nt[g] == 0) continue;
-        const int st = kTA * g + (int)wg;
+        if (!tok_valid[g] || tok_nt[g] == 0) continue;
+        const int st = ST(g);
         const int kk = min(a.k, tok_t[g] + 1);
         const uint32_t c0 = sCnt[st * 4], c1 = sCnt[st * 4 + 1], c2 = sCnt[st * 4 + 2], c3 = sCnt[st * 4 + 3];
         const int m = (int)(c0 + c1 + c2 + c3);
