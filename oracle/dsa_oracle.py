@@ -44,6 +44,7 @@ __all__ = [
     "causal_topk_row",
     "indexer_topk",
     "selection_stats_row",
+    "selection_recall_row",
     "sparse_attention_row",
     "sparse_attention",
     "decode_indexer_topk",
@@ -175,6 +176,20 @@ def selection_stats_row(scores_row, t: int, k: int) -> dict:
         "margin": float(tau - nxt),
         "max_abs": float(np.max(np.abs(s))),
     }
+
+
+def selection_recall_row(teacher_row, student_row) -> float:
+    """Set recall R = |T ∩ S| / |T| of a student selection S against a teacher
+    selection T, eq. (14) of the DSA page §3.1 (there |T| = k; for a row with
+    t + 1 <= k both sets hold its t + 1 positions, so |T| is the count of
+    valid teacher entries).  Entries < 0 are unused slots; slot order is
+    irrelevant.  A row with an empty teacher set has recall 1.
+    """
+    t = {int(x) for x in np.asarray(teacher_row).ravel() if x >= 0}
+    s = {int(x) for x in np.asarray(student_row).ravel() if x >= 0}
+    if not t:
+        return 1.0
+    return len(t & s) / len(t)
 
 
 def indexer_topk(q, k, w, topk: int, q_offset: int = 0, rows=None) -> np.ndarray:

@@ -347,3 +347,24 @@ def test_decode_equals_last_prefill_row():
         assert pre[0, L - 1].tolist() == idx[b].tolist()
         o2, l2 = O.sparse_attention_row(q[b], lat[lo:lo + L], idx[b], 0.4, Dv)
         assert np.allclose(out[b], o2) and np.allclose(lse[b], l2)
+
+
+def test_selection_recall_pins():
+    # eq. (14): R = |T ∩ S| / |T|, order-free, unused slots ignored
+    assert O.selection_recall_row([0, 1, 2, 3], [3, 2, 1, 0]) == 1.0
+    assert O.selection_recall_row([0, 1, 2, 3], [4, 5, 6, 7]) == 0.0
+    assert O.selection_recall_row([0, 1, 2, 3], [1, 3, 8, 9]) == 0.5
+    assert O.selection_recall_row([5, 2, -1, -1], [2, 7, -1, -1]) == 0.5
+    assert O.selection_recall_row([-1, -1], [3, -1]) == 1.0
+    # the worked example's top-2 {0, 1} against a selector that swapped in position 2
+    ex = _worked()
+    s = np.array(ex["scores"], dtype=float)
+    teacher = O.causal_topk_row(s, 2, 2)
+    assert O.selection_recall_row(teacher, [0, 2]) == 0.5
+    # brute force on random sets: the definition written out with loops
+    rng = np.random.default_rng(5)
+    for _ in range(50):
+        a = rng.choice(40, size=10, replace=False)
+        b = rng.choice(40, size=10, replace=False)
+        hits = sum(1 for x in a for y in b if x == y)
+        assert O.selection_recall_row(a, b) == hits / 10
