@@ -166,7 +166,7 @@ class PrefillRun:
     def __init__(self, w: W.Workload, device):
         import learned_token_indexer_b200 as dsa
         self.dsa, self.w, self.dev = dsa, w, device
-        self.d = W.make_prefill_inputs(w, device)
+        self.d = W.make_prefill_inputs(w, device, keep_bf16=w.fp8)
         self.ws_idx = dsa.Workspace(device)
         self.ws_att = dsa.Workspace(device)
         self.idx = torch.empty((w.B, w.n, w.k), dtype=torch.int32, device=device)
@@ -208,6 +208,31 @@ class PrefillRun:
 
     def rows(self):
         return self.w.B * self.w.n
+
+    def selection_diagnostics(self):
+        """FP8 indexer only (outside the timed region): the set recall
+        R = |T ∩ S| / |T| (eq. (14)) of this step's e4m3 selection S against
+        the bf16 selection T of the same draws, over rows with t + 1 > k."""
+        w, d, dsa = self.w, self.d, self.dsa
+        if not w.fp8 or "qI_bf16" not in d:
+            return None
+        ref = torch.empty_like(self.idx)
+        ws = dsa.Workspace(self.dev)
+        for c0 in range(0, w.n, self.chunk):
+            c1 = min(w.n, c0 + self.chunk)
+            sl = (slice(None), slice(c0, c1))
+            dsa.indexer_topk_prefill(d["qI_bf16"][sl], d["kI_bf16"], d["w"][sl], w.k, q_offset=c0, idx_out=ref[sl],
+                                     workspace=ws)
+        inter, cnt = dsa.selection_overlap(ref, self.idx, w.n, return_counts=True)
+        torch.cuda.synchronize()
+        ws.check()
+        rec = (inter.float() / cnt.clamp(min=1).float())[:, w.k:].flatten()
+        q = torch.quantile(rec, torch.tensor([0.01, 0.5], device=rec.device))
+        return {"fp8_vs_bf16_recall": {"mean": round(float(rec.mean()), 5), "p01": round(float(q[0]), 5),
+                                       "median": round(float(q[1]), 5), "min": round(float(rec.min()), 5),
+                                       "rows": int(rec.numel()),
+                                       "definition": "|T ∩ S| / |T|, T = bf16 selection of the same draws, "
+                                                     "S = e4m3 selection; rows with t + 1 > k"}}
 
     def kernel_work(self):
         w = self.w
@@ -536,6 +561,9 @@ def run_b200(args):
     }
     if e2e is not None:
         line["e2e"] = e2e
+    diag = run.selection_diagnostics() if hasattr(run, "selection_diagnostics") else None
+    if diag:
+        line["diagnostics"] = diag
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_budget)
     print(json.dumps(line), flush=True)

@@ -200,6 +200,21 @@ dsa_status dsa_topk_rows(int rows, int ncols, int64_t row_stride, const float* s
                          void* stream);
 dsa_status dsa_selftest_bounded_wait(uint64_t timeout_ns, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Selection diagnostic (§3.1, eq. (14)): the set recall of a student
+ * selection S against a teacher selection T is R = |T ∩ S| / k.  For each
+ * of `rows` rows of two index arrays idx_a (teacher) and idx_b (student),
+ * both [rows, k] int32 (positions, -1 = unused; slot order irrelevant):
+ *   inter_out[r]   = |valid(A_r) ∩ valid(B_r)|     (int32, [rows])
+ *   count_a_out[r] = |valid(A_r)|                  (int32, [rows], or NULL)
+ * so R_r = inter_out[r] / count_a_out[r] (= / k when every row holds k).
+ * Positions outside [0, max_pos) are not counted.  max_pos <= 2^20.
+ * A row's positions must be distinct within each array (true of every
+ * selection this library produces).  Needs no workspace.
+ * ---------------------------------------------------------------------- */
+dsa_status dsa_selection_overlap(int rows, int k, int max_pos, const int32_t* idx_a, const int32_t* idx_b,
+                                 int32_t* inter_out, int32_t* count_a_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -228,6 +228,20 @@ def sparse_attn_decode(q, latent_cache, cu_seqlens, idx, dv: int, total_len: int
     return (out, lse) if lse is not None else out
 
 
+def selection_overlap(idx_teacher, idx_student, max_pos: int, return_counts: bool = False):
+    """Per-row |T ∩ S| of two [rows, k] int32 selections on the device (the
+    numerator of the set recall R_k, eq. (14)); with return_counts also
+    |T| per row.  Recall = inter / count."""
+    k = idx_teacher.shape[-1]
+    rows = idx_teacher.numel() // k
+    dev = idx_teacher.device
+    inter = torch.empty(idx_teacher.shape[:-1], dtype=torch.int32, device=dev)
+    count = torch.empty_like(inter) if return_counts else None
+    _check(lib().dsa_selection_overlap(rows, k, int(max_pos), _ptr(idx_teacher), _ptr(idx_student), _ptr(inter),
+                                       _ptr(count), _stream(dev)))
+    return (inter, count) if return_counts else inter
+
+
 # --------------------------------------------------------------------------
 # Debug / test
 # --------------------------------------------------------------------------

@@ -30,6 +30,7 @@ SIGNATURES = {
     "dsa_indexer_scores": (_i, [_i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "dsa_topk_rows": (_i, [_i, _i, _i64, _p, _p, _i, _p, _p, _p, _sz, _p]),
     "dsa_selftest_bounded_wait": (_i, [_u64, _p, _sz, _p]),
+    "dsa_selection_overlap": (_i, [_i, _i, _i, _p, _p, _p, _p, _p]),
 }
 
 _lib = None

@@ -464,4 +464,18 @@ dsa_status dsa_selftest_bounded_wait(uint64_t timeout_ns, void* workspace, size_
   return DSA_OK;
 }
 
+// ---------------------------------------------------------------- diagnostics
+dsa_status dsa_selection_overlap(int rows, int k, int max_pos, const int32_t* idx_a, const int32_t* idx_b,
+                                 int32_t* inter_out, int32_t* count_a_out, void* stream) {
+  DSA_CHECK(rows >= 0 && k >= 1 && max_pos >= 1, DSA_ERR_INVALID_ARG, "need rows >= 0, k >= 1, max_pos >= 1");
+  DSA_CHECK(max_pos <= (1 << 20), DSA_ERR_UNSUPPORTED, "max_pos above 2^20 (the row bitmap lives in shared memory)");
+  DSA_CHECK(idx_a && idx_b && inter_out, DSA_ERR_INVALID_ARG, "null tensor pointer");
+  if (rows == 0) return DSA_OK;
+  const int grid = std::min(rows, 4 * sm_count());
+  cudaError_t e = dsa::launch_selection_overlap(rows, k, max_pos, idx_a, idx_b, inter_out, count_a_out, grid,
+                                                (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "selection_overlap launch");
+  return DSA_OK;
+}
+
 }  // extern "C"

@@ -89,6 +89,8 @@ cudaError_t launch_fill_trivial_rows(int B, int nq, int q_offset, int rows_per_s
 cudaError_t launch_fill_f32(float* p, int64_t n, float v, cudaStream_t stream);
 cudaError_t launch_sparse_attn(const AttnArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_wait_selftest(DeviceStatus* status, uint64_t timeout_ns, cudaStream_t stream);
+cudaError_t launch_selection_overlap(int rows, int k, int max_pos, const int32_t* idx_a, const int32_t* idx_b,
+                                     int32_t* inter, int32_t* count_a, int grid, cudaStream_t stream);
 
 // Host helpers implemented in api.cu.
 void set_last_error(const char* msg);                 // message returned by dsa_last_error()

@@ -214,4 +214,76 @@ cudaError_t launch_wait_selftest(DeviceStatus* status, uint64_t timeout_ns, cuda
   return cudaGetLastError();
 }
 
+
+// ---------------------------------------------------------------------------
+// Selection diagnostic: per row, how many valid entries of selection A also
+// appear in selection B (the numerator of the set recall R_k = |T ∩ S| / k,
+// eq. (14) of the same page, §3.1), and how many valid entries A has.  One
+// row at a time per CTA: A's positions go into a shared-memory bitmap of
+// max_pos bits, then B's entries are tested against it.  Slot order and -1
+// slots are irrelevant; entries outside [0, max_pos) are not counted.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int kOverlapThreads = 256;
+}
+
+__global__ void __launch_bounds__(kOverlapThreads) selection_overlap_kernel(int rows, int k, int max_pos,
+                                                                            const int32_t* idx_a,
+                                                                            const int32_t* idx_b, int32_t* inter,
+                                                                            int32_t* count_a) {
+  extern __shared__ uint32_t bits[];
+  __shared__ uint32_t s_inter, s_count;
+  const int words = (max_pos + 31) / 32;
+  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+    for (int i = threadIdx.x; i < words; i += kOverlapThreads) bits[i] = 0u;
+    if (threadIdx.x == 0) {
+      s_inter = 0u;
+      s_count = 0u;
+    }
+    __syncthreads();
+    const int32_t* a = idx_a + (int64_t)r * k;
+    const int32_t* b = idx_b + (int64_t)r * k;
+    uint32_t na = 0;
+    for (int j = threadIdx.x; j < k; j += kOverlapThreads) {
+      const int p = a[j];
+      if (p >= 0 && p < max_pos) {
+        atomicOr(&bits[p >> 5], 1u << (p & 31));
+        ++na;
+      }
+    }
+    __syncthreads();
+    uint32_t hit = 0;
+    for (int j = threadIdx.x; j < k; j += kOverlapThreads) {
+      const int p = b[j];
+      if (p >= 0 && p < max_pos && (bits[p >> 5] >> (p & 31)) & 1u) ++hit;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      hit += __shfl_xor_sync(0xffffffffu, hit, o);
+      na += __shfl_xor_sync(0xffffffffu, na, o);
+    }
+    if ((threadIdx.x & 31u) == 0u) {
+      atomicAdd(&s_inter, hit);
+      atomicAdd(&s_count, na);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      inter[r] = (int32_t)s_inter;
+      if (count_a) count_a[r] = (int32_t)s_count;
+    }
+    __syncthreads();   // the bitmap is cleared for the next row
+  }
+}
+
+cudaError_t launch_selection_overlap(int rows, int k, int max_pos, const int32_t* idx_a, const int32_t* idx_b,
+                                     int32_t* inter, int32_t* count_a, int grid, cudaStream_t stream) {
+  if (rows == 0) return cudaSuccess;
+  const size_t smem = (size_t)((max_pos + 31) / 32) * 4;
+  cudaError_t e = cudaFuncSetAttribute(selection_overlap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  selection_overlap_kernel<<<grid, kOverlapThreads, smem, stream>>>(rows, k, max_pos, idx_a, idx_b, inter, count_a);
+  return cudaGetLastError();
+}
+
 }  // namespace dsa

@@ -98,7 +98,7 @@ def quantize_fp8_per_token(x: torch.Tensor, group_dims: int):
 
 
 def make_prefill_inputs(w: Workload, device="cpu", n: Optional[int] = None,
-                        with_attention: bool = True) -> dict:
+                        with_attention: bool = True, keep_bf16: bool = False) -> dict:
     """All inputs of one prefill workload (whole sequence; chunks are views).
 
     Returns a dict of tensors on ``device``:
@@ -106,6 +106,8 @@ def make_prefill_inputs(w: Workload, device="cpu", n: Optional[int] = None,
       kI [B,n,dI]    bf16 (or e4m3 codes + k_scale [B,n]),
       w  [B,n,HI]    fp32,
       q  [B,n,H,Dqk] bf16, latent [B,n,Dqk] bf16  (if with_attention).
+    FP8 workloads with keep_bf16 also return qI_bf16 / kI_bf16: the same
+    draws rounded to bf16 instead of quantised (a reference selection).
     """
     n = w.n if n is None else n
     g = _gen(device, w.seed)
@@ -120,6 +122,9 @@ def make_prefill_inputs(w: Workload, device="cpu", n: Optional[int] = None,
         if w.fp8:
             out["qI"], out["q_scale"] = quantize_fp8_per_token(qI, 2)
             out["kI"], out["k_scale"] = quantize_fp8_per_token(kI, 1)
+            if keep_bf16:
+                out["qI_bf16"] = qI.to(torch.bfloat16)
+                out["kI_bf16"] = kI.to(torch.bfloat16)
         else:
             out["qI"] = qI.to(torch.bfloat16)
             out["kI"] = kI.to(torch.bfloat16)

@@ -406,3 +406,29 @@ def test_attention_full_prefill_sampled():
     torch.cuda.synchronize()
     _no_device_errors(ws)
     _attn_check(d["q"], d["latent"], idx, out, lse, w.scale, w.Dv, W.sample_rows(w, 128))
+
+
+# --------------------------------------------------------------------------
+# selection diagnostic (eq. (14))
+# --------------------------------------------------------------------------
+
+def test_selection_overlap_matches_oracle_recall():
+    g = torch.Generator().manual_seed(14)
+    rows, k, max_pos = 40, 64, 300
+    a = torch.stack([torch.randperm(max_pos, generator=g)[:k] for _ in range(rows)]).int()
+    b = torch.stack([torch.randperm(max_pos, generator=g)[:k] for _ in range(rows)]).int()
+    b[:5] = a[:5].flip(-1)                      # identical sets in another order
+    for r in range(5, 10):                      # half shared, positions distinct within the row
+        keep = a[r, : k // 2]
+        rest = [int(x) for x in torch.randperm(max_pos, generator=g) if int(x) not in set(keep.tolist())]
+        b[r] = torch.cat([keep, torch.tensor(rest[: k - k // 2], dtype=torch.int32)])
+    a[10:15, 40:] = -1                          # short rows padded with -1
+    b[15:20] = -1                               # empty student
+    a[20:25] = -1                               # empty teacher
+    inter, cnt = dsa.selection_overlap(a.cuda(), b.cuda(), max_pos, return_counts=True)
+    torch.cuda.synchronize()
+    inter, cnt = inter.cpu().numpy(), cnt.cpu().numpy()
+    for r in range(rows):
+        assert cnt[r] == int((a[r] >= 0).sum())
+        rec = inter[r] / cnt[r] if cnt[r] else 1.0
+        assert rec == O.selection_recall_row(a[r].numpy(), b[r].numpy()), r
