@@ -6,8 +6,9 @@ module.  The CUDA library never calls it, and it shares no code, constant or
 helper with the CUDA library.
 
 Source: the page "2.2.1 · DSA 与索引器: 先召回 token, 再计算 Sparse MLA"
-(called "the DSA page" below), §1.1 eqs. (1)-(6), §2 (decode, quantised
-indexer key cache) and §3.1 eq. (18), §3.2 eqs. (19)-(20).
+(called "the DSA page" below), §1.1 eqs. (1)-(6), §1.2 eqs. (8) and (16)
+(sparse-stage indexer KL and its teacher), §2 (decode, quantised indexer key
+cache) and §3.1 eqs. (14), (18), §3.2 eqs. (19)-(20).
 
 Everything is float64 numpy.  Inputs are converted exactly to float64 first:
 bf16 values are exact in float64, and FP8-e4m3 codes are decoded by
@@ -23,11 +24,20 @@ Readings of points the page leaves open (each is repeated where it is used):
     whole latent row and the value is its first ``Dv`` columns; the rotary
     part of query and latent arrives already rotated;
   * a decode step's query is the last token of its sequence (position L-1)
-    and it scans all L cached keys, itself included.
+    and it scans all L cached keys, itself included;
+  * eq. (8): teacher weights arrive per slot of the index tensor and are
+    divided by their sum over the valid slots (the retained mass); a row with
+    no valid slot or zero retained mass has loss 0 and zero gradient;
+    0 * log 0 = 0; the ReLU of eq. (1) has derivative 0 at 0;
+  * the sparse-stage teacher sums the heads' attention probabilities over the
+    selected set and L1-normalises the sum (eq. (16) with the aggregation
+    the DSA report uses: sum over heads, then L1 along the sequence).
 
 Parity status: every function here is pinned by ``tests/test_oracle.py``
 (worked example of §1.1, the min(k, t+1) rule, brute force on tiny inputs,
-library special cases, and the invariants of §3.1/§3.2).
+library special cases, the invariants of §3.1/§3.2, and for eq. (8) the
+worked example's KL, torch's kl_div and central finite differences of the
+loss for every gradient).
 """
 
 from __future__ import annotations
@@ -49,6 +59,10 @@ __all__ = [
     "sparse_attention",
     "decode_indexer_topk",
     "decode_sparse_attention",
+    "attention_teacher_row",
+    "attention_teacher",
+    "indexer_kl_sparse_row",
+    "indexer_kl_sparse",
 ]
 
 
@@ -311,6 +325,140 @@ def decode_sparse_attention(q, latent_cache, cu_seqlens, idx, scale: float, dv: 
         lo, hi = int(cu[b]), int(cu[b + 1])
         out[b], lse[b] = sparse_attention_row(q[b], latent_cache[lo:hi], idx[b], scale, dv)
     return out, lse
+
+
+# ---------------------------------------------------------------------------
+# Eq. (8): sparse-stage indexer KL on the selected set, and its teacher
+# ---------------------------------------------------------------------------
+
+def attention_teacher_row(q_t, latent, sel, scale: float) -> np.ndarray:
+    """Teacher distribution of token t over its selected set, taken from the
+    sparse main attention (DSA page §1.2, the remark after eq. (8), and
+    eq. (16) with the DSA report's aggregation).
+
+    For every query head h the attention probabilities over the selected set,
+    a_h[s] = softmax_s(scale * q_t[h] . c_s), are recomputed from scratch;
+    they are summed over the heads and the sum is L1-normalised along the
+    selected positions.  Returns one weight per slot of ``sel`` (0 in the
+    unused slots, which hold -1); all zeros if no slot is valid.
+    """
+    q_t = _f64(q_t)
+    latent = _f64(latent)
+    sel = np.asarray(sel, dtype=np.int64)
+    out = np.zeros(sel.shape[0])
+    valid = sel >= 0
+    if not valid.any():
+        return out
+    c = latent[sel[valid]]                           # [m, Dqk]
+    z = scale * (q_t @ c.T)                          # [H, m]
+    e = np.exp(z - z.max(axis=1, keepdims=True))
+    a = e / e.sum(axis=1, keepdims=True)             # per-head softmax over S_t
+    p = a.sum(axis=0)                                # sum over heads
+    out[valid] = p / p.sum()                         # L1 normalisation
+    return out
+
+
+def attention_teacher(q, latent, idx, scale: float, rows=None) -> np.ndarray:
+    """``attention_teacher_row`` for a prefill chunk.
+
+    q: [B, nq, H, Dqk], latent: [B, kv_len, Dqk], idx: [B, nq, k].
+    Returns [B, nq, k] float64 (NaN in rows left out by ``rows``).
+    """
+    q = _f64(q)
+    latent = _f64(latent)
+    idx = np.asarray(idx.cpu() if hasattr(idx, "cpu") else idx, dtype=np.int64)
+    B, nq, k = idx.shape
+    out = np.full((B, nq, k), np.nan)
+    todo = rows if rows is not None else [(b, i) for b in range(B) for i in range(nq)]
+    for b, i in todo:
+        out[b, i] = attention_teacher_row(q[b, i], latent[b], idx[b, i], scale)
+    return out
+
+
+def indexer_kl_sparse_row(q_t, k_all, w_t, sel, teacher, grad_scale: float = 1.0) -> dict:
+    """Eq. (8) of the DSA page for one token t, with its gradient.
+
+        KL_t = D_KL( p_{t,S_t} || Softmax(I_{t,S_t}) )
+
+    Steps, in the page's order:
+      1. the teacher's weights on the selected slots are divided by their
+         sum (the retained mass), so both sides are distributions over S_t;
+      2. the indexer scores I_{t,s} of eq. (1) are recomputed for s in S_t;
+      3. the student is the softmax of those scores over S_t;
+      4. KL_t = sum_s p_s (log p_s - log softmax(I)_s), with 0 log 0 = 0.
+    Backward, for a loss L with dL/dKL_t = grad_scale:
+      g_s  = dL/dI_s = grad_scale * (softmax(I)_s - p_s)
+      dw_j = sum_s g_s ReLU(d_sj),             d_sj = q_t[j] . k_s
+      dq_j = sum_s g_s w_j [d_sj > 0] k_s       (ReLU'(0) = 0)
+      dk_s = sum_j g_s w_j [d_sj > 0] q_t[j]
+
+    q_t: [H_I, d_I]; k_all: [kv_len, d_I]; w_t: [H_I]; sel: [k] positions
+    (-1 = unused slot; the valid ones are distinct); teacher: [k] weights
+    >= 0.  Returns kl (float), grad_logits [k] (0 in unused slots),
+    dq [H_I, d_I], dw [H_I] and dk [k, d_I] (row r is the gradient of key
+    sel[r]; zero rows for unused slots).
+    """
+    q_t = _f64(q_t)
+    k_all = _f64(k_all)
+    w_t = _f64(w_t)
+    sel = np.asarray(sel, dtype=np.int64)
+    teacher = _f64(teacher)
+    K = sel.shape[0]
+    HI, dI = q_t.shape
+    res = {"kl": 0.0, "grad_logits": np.zeros(K), "dq": np.zeros((HI, dI)),
+           "dw": np.zeros(HI), "dk": np.zeros((K, dI))}
+    valid = sel >= 0
+    if not valid.any():
+        return res
+    p = teacher[valid]
+    mass = p.sum()
+    if not mass > 0.0:
+        return res
+    p_hat = p / mass                                  # step 1
+    kS = k_all[sel[valid]]                            # [m, d_I]
+    dots = kS @ q_t.T                                 # [m, H_I]
+    scores = np.maximum(dots, 0.0) @ w_t              # step 2, eq. (1)
+    top = scores.max()
+    log_z = top + math.log(np.exp(scores - top).sum())
+    log_student = scores - log_z                      # step 3
+    pos = p_hat > 0.0
+    res["kl"] = float(np.sum(p_hat[pos] * (np.log(p_hat[pos]) - log_student[pos])))   # step 4
+    g = grad_scale * (np.exp(log_student) - p_hat)
+    G = g[:, None] * w_t[None, :] * (dots > 0.0)      # dL/d d_sj
+    res["grad_logits"][valid] = g
+    res["dw"] = (np.maximum(dots, 0.0) * g[:, None]).sum(axis=0)
+    res["dq"] = G.T @ kS
+    res["dk"][valid] = G @ q_t
+    return res
+
+
+def indexer_kl_sparse(q, k, w, idx, teacher, grad_scale: float = 1.0, rows=None) -> dict:
+    """Eq. (8) summed over the rows of a prefill chunk, with gradients.
+
+    q: [B, nq, H_I, d_I], k: [B, kv_len, d_I], w: [B, nq, H_I],
+    idx: [B, nq, topk], teacher: [B, nq, topk].  Returns kl [B, nq],
+    grad_logits [B, nq, topk], dq, dw (shapes of q and w) and dk [B, kv_len,
+    d_I], the sum over rows of each selected key's gradient.  ``rows``
+    restricts the work to a list of (b, i) rows (the others stay 0).
+    """
+    q = _f64(q)
+    k = _f64(k)
+    w = _f64(w)
+    teacher = _f64(teacher)
+    idx = np.asarray(idx.cpu() if hasattr(idx, "cpu") else idx, dtype=np.int64)
+    B, nq, topk = idx.shape
+    out = {"kl": np.zeros((B, nq)), "grad_logits": np.zeros((B, nq, topk)),
+           "dq": np.zeros(q.shape), "dw": np.zeros(w.shape), "dk": np.zeros(k.shape)}
+    todo = rows if rows is not None else [(b, i) for b in range(B) for i in range(nq)]
+    for b, i in todo:
+        r = indexer_kl_sparse_row(q[b, i], k[b], w[b, i], idx[b, i], teacher[b, i], grad_scale)
+        out["kl"][b, i] = r["kl"]
+        out["grad_logits"][b, i] = r["grad_logits"]
+        out["dq"][b, i] = r["dq"]
+        out["dw"][b, i] = r["dw"]
+        v = idx[b, i] >= 0
+        np.add.at(out["dk"][b], idx[b, i][v], r["dk"][v])
+    return out
 
 
 def softmax_scale_default(dqk: int) -> float:

@@ -368,3 +368,196 @@ def test_selection_recall_pins():
         b = rng.choice(40, size=10, replace=False)
         hits = sum(1 for x in a for y in b if x == y)
         assert O.selection_recall_row(a, b) == hits / 10
+
+
+# --------------------------------------------------------------------------
+# Eq. (8): sparse-stage indexer KL and the sparse-attention teacher (§1.2)
+# --------------------------------------------------------------------------
+
+def _example_kl_inputs(g):
+    q = np.array(g["q"], float)
+    keys = np.array(g["keys"], float)
+    w = np.array(g["w"], float)
+    sel = np.array(g["selected_positions_0based"] + [-1])      # width 3, one unused slot
+    return q, keys, w, sel
+
+
+def test_kl_worked_example_teacher_and_loss():
+    """The printed example: the selector keeps 1-based positions 1 and 2 with
+    indexer scores 1.5 and 1.5 (eqs. (5)-(6)), while the main attention puts
+    weights of about 0.269 / 0.731 on them.  With one attention head the
+    sparse-attention teacher is exactly those weights, and the student is
+    uniform, so KL = ln 2 - H(p) (a closed form, not the oracle's sum)."""
+    g = _worked()
+    qa, latent = _example_attention_inputs(g)
+    sel = np.array(g["selected_positions_0based"] + [-1])
+    p = O.attention_teacher_row(qa, latent, sel, 1.0)
+    tol = 0.5 * 10 ** -g["printed_decimals"]
+    assert np.allclose(p[:2], g["attention_weights_printed"], atol=tol, rtol=0)
+    assert p[2] == 0.0
+    q, keys, w, sel = _example_kl_inputs(g)
+    r = O.indexer_kl_sparse_row(q, keys, w, sel, p)
+    a = np.array(g["attention_logits"])
+    pa = np.exp(a) / np.exp(a).sum()
+    entropy = -(pa * np.log(pa)).sum()
+    assert abs(r["kl"] - (math.log(2.0) - entropy)) < 1e-12
+    # the gradient with respect to the scores is student - teacher = 0.5 - p
+    assert np.allclose(r["grad_logits"], [0.5 - pa[0], 0.5 - pa[1], 0.0], atol=1e-12, rtol=0)
+    # with the printed (rounded) weights the loss agrees to the rounding
+    r2 = O.indexer_kl_sparse_row(q, keys, w, sel, np.array(g["attention_weights_printed"] + [0.0]))
+    assert abs(r2["kl"] - r["kl"]) < 2e-3
+
+
+def test_kl_dense_subvector_is_renormalised_by_retained_mass():
+    """Remark after eq. (8): a teacher cut out of a dense distribution is divided
+    by its retained mass.  The page's miss case gives position 3 a full logit
+    of 2.0; the dense softmax's sub-vector on {1, 2} must give the same loss
+    as the sparse-attention teacher on that set."""
+    g = _worked()
+    q, keys, w, sel = _example_kl_inputs(g)
+    a = np.array(g["attention_logits"] + [g["miss_case_logit_position3"]])
+    dense = np.exp(a) / np.exp(a).sum()
+    sub = np.array([dense[0], dense[1], 0.0])
+    assert sub.sum() < 0.5                         # most mass is outside the set
+    qa, latent = _example_attention_inputs(g)
+    p = O.attention_teacher_row(qa, latent, sel, 1.0)
+    r_sub = O.indexer_kl_sparse_row(q, keys, w, sel, sub)
+    r_p = O.indexer_kl_sparse_row(q, keys, w, sel, p)
+    assert abs(r_sub["kl"] - r_p["kl"]) < 1e-12
+    for key in ("grad_logits", "dq", "dw", "dk"):
+        assert np.allclose(r_sub[key], r_p[key], atol=1e-12, rtol=0)
+
+
+def _kl_case(rng, HI=3, dI=5, kv_len=11, k=8, n_valid=6):
+    q = rng.standard_normal((HI, dI))
+    keys = rng.standard_normal((kv_len, dI))
+    w = rng.standard_normal(HI)
+    sel = np.full(k, -1)
+    sel[:n_valid] = rng.choice(kv_len, n_valid, replace=False)
+    perm = rng.permutation(k)                      # unused slots anywhere
+    sel = sel[perm]
+    teacher = np.where(sel >= 0, rng.random(k) + 0.05, 0.0)
+    return q, keys, w, sel, teacher
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_kl_matches_torch_kl_div(seed):
+    rng = np.random.default_rng(100 + seed)
+    q, keys, w, sel, teacher = _kl_case(rng)
+    r = O.indexer_kl_sparse_row(q, keys, w, sel, teacher)
+    v = sel >= 0
+    scores = torch.from_numpy(O.indexer_scores_row(q, keys[sel[v]], w))     # eq. (1), pinned above
+    target = torch.from_numpy(teacher[v] / teacher[v].sum())
+    ref = torch.nn.functional.kl_div(torch.log_softmax(scores, 0), target, reduction="sum")
+    assert abs(r["kl"] - float(ref)) < 1e-12
+    assert r["kl"] >= 0.0
+
+
+def test_kl_is_zero_when_teacher_equals_student():
+    rng = np.random.default_rng(7)
+    q, keys, w, sel, _ = _kl_case(rng)
+    v = sel >= 0
+    teacher = np.zeros(sel.shape[0])
+    teacher[v] = 3.0 * np.exp(O.indexer_scores_row(q, keys[sel[v]], w))   # unnormalised on purpose
+    r = O.indexer_kl_sparse_row(q, keys, w, sel, teacher)
+    assert abs(r["kl"]) < 1e-14
+    for key in ("grad_logits", "dq", "dw", "dk"):
+        assert np.abs(r[key]).max() < 1e-14
+
+
+def test_kl_invariances_and_degenerate_rows():
+    rng = np.random.default_rng(8)
+    q, keys, w, sel, teacher = _kl_case(rng)
+    r = O.indexer_kl_sparse_row(q, keys, w, sel, teacher)
+    # the teacher's scale does not matter (it is renormalised over S_t)
+    r2 = O.indexer_kl_sparse_row(q, keys, w, sel, 4.25 * teacher)
+    assert abs(r2["kl"] - r["kl"]) < 1e-12
+    # the slot order does not matter
+    perm = rng.permutation(sel.shape[0])
+    r3 = O.indexer_kl_sparse_row(q, keys, w, sel[perm], teacher[perm])
+    assert abs(r3["kl"] - r["kl"]) < 1e-12
+    assert np.allclose(r3["dq"], r["dq"], atol=1e-12) and np.allclose(r3["dw"], r["dw"], atol=1e-12)
+    assert np.allclose(r3["dk"], r["dk"][perm], atol=1e-12)
+    assert np.allclose(r3["grad_logits"], r["grad_logits"][perm], atol=1e-12)
+    # the score gradient is a difference of two distributions: it sums to 0
+    assert abs(r["grad_logits"].sum()) < 1e-12
+    # grad_scale multiplies every gradient, not the loss
+    r4 = O.indexer_kl_sparse_row(q, keys, w, sel, teacher, grad_scale=0.5)
+    assert r4["kl"] == r["kl"] and np.allclose(r4["dq"], 0.5 * r["dq"], atol=1e-15)
+    # no valid slot, or a teacher with no mass on S_t: loss and gradients are 0
+    for s, t in ((np.full(8, -1), teacher), (sel, np.zeros(8))):
+        e = O.indexer_kl_sparse_row(q, keys, w, s, t)
+        assert e["kl"] == 0.0 and not np.any(e["dq"]) and not np.any(e["dk"]) and not np.any(e["dw"])
+    # a single valid slot: the student and the teacher are both a point mass
+    one = np.full(8, -1)
+    one[3] = 5
+    e = O.indexer_kl_sparse_row(q, keys, w, one, teacher + 1.0)
+    assert e["kl"] == 0.0 and np.abs(e["dq"]).max() == 0.0
+
+
+def _central_difference(f, x, h=1e-6):
+    grad = np.zeros_like(x)
+    it = np.nditer(x, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        old = x[i]
+        x[i] = old + h
+        fp = f()
+        x[i] = old - h
+        fm = f()
+        x[i] = old
+        grad[i] = (fp - fm) / (2 * h)
+    return grad
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_kl_gradients_match_finite_differences(seed):
+    """Every analytic gradient of eq. (8) against a central difference of the
+    summed loss, on a 2-sequence chunk whose rows share keys (so dk sums
+    over rows).  Inputs keep every q.k at least 1e-3 away from the ReLU kink."""
+    rng = np.random.default_rng(200 + seed)
+    B, nq, kv_len, HI, dI, k, gs = 2, 3, 9, 3, 4, 6, 0.7
+    while True:
+        q = rng.standard_normal((B, nq, HI, dI))
+        kk = rng.standard_normal((B, kv_len, dI))
+        if np.abs(np.einsum("bnhd,bsd->bnhs", q, kk)).min() > 1e-3:
+            break
+    w = rng.standard_normal((B, nq, HI))
+    idx = np.full((B, nq, k), -1)
+    for b in range(B):
+        for i in range(nq):
+            m = [6, 4, 1][i]
+            idx[b, i, :m] = rng.choice(kv_len, m, replace=False)
+    teacher = np.where(idx >= 0, rng.random((B, nq, k)) + 0.1, 0.0)
+    res = O.indexer_kl_sparse(q, kk, w, idx, teacher, grad_scale=gs)
+
+    def loss():
+        return gs * O.indexer_kl_sparse(q, kk, w, idx, teacher)["kl"].sum()
+
+    for name, x in (("dq", q), ("dw", w), ("dk", kk)):
+        num = _central_difference(loss, x)
+        assert np.allclose(res[name], num, atol=1e-7, rtol=1e-6), name
+    # keys nobody selected get no gradient
+    used = np.zeros((B, kv_len), bool)
+    for b in range(B):
+        used[b, idx[b][idx[b] >= 0]] = True
+    assert not np.any(res["dk"][~used])
+
+
+def test_attention_teacher_reproduces_the_mean_head_output():
+    """Sum over heads then L1 normalisation (eq. (16) with the DSA report's
+    aggregation): with every head normalised, p @ C must equal the mean over
+    heads of the eq. (3) output (pinned above against scaled_dot_product_attention)
+    when the value is the whole latent row; the latent rows are linearly
+    independent, so this fixes p."""
+    rng = np.random.default_rng(9)
+    H, Dqk, kv_len, k = 4, 16, 12, 8
+    q = rng.standard_normal((H, Dqk))
+    latent = rng.standard_normal((kv_len, Dqk))
+    sel = np.array([3, -1, 7, 0, 11, -1, 5, 9])
+    p = O.attention_teacher_row(q, latent, sel, 0.3)
+    v = sel >= 0
+    assert np.all(p[~v] == 0.0) and abs(p.sum() - 1.0) < 1e-12 and np.all(p[v] > 0)
+    out, _ = O.sparse_attention_row(q, latent, sel, 0.3, Dqk)
+    assert np.allclose(p[v] @ latent[sel[v]], out.mean(axis=0), atol=1e-12, rtol=0)
+    assert not np.any(O.attention_teacher_row(q, latent, np.full(5, -1), 0.3))
