@@ -215,6 +215,47 @@ dsa_status dsa_selftest_bounded_wait(uint64_t timeout_ns, void* workspace, size_
 dsa_status dsa_selection_overlap(int rows, int k, int max_pos, const int32_t* idx_a, const int32_t* idx_b,
                                  int32_t* inter_out, int32_t* count_a_out, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Sparse-stage indexer loss (§1.2, eq. (8)), forward and backward.
+ * In the sparse training stage the indexer is fitted, for every token t,
+ * by KL_t = D_KL(p_{t,S_t} || Softmax(I_{t,S_t})) on the selected set S_t
+ * only; both sides are distributions over S_t (the teacher's weights are
+ * divided by their retained mass, the remark after eq. (8)), and I are the
+ * eq. (1) scores recomputed on S_t.  The indexer's inputs are detached from
+ * the main model, so this loss alone trains the indexer (§1.2).
+ *
+ *   rows (b, i), i < nq, of a chunk; positions index the sequence's keys.
+ *   qI      [B, nq, HI, dI] bf16      kI [B, kv_len, dI] bf16
+ *   w       [B, nq, HI]     fp32      idx [B, nq, k] int32 positions in
+ *                                     [0, kv_len) or -1 (unused slot);
+ *                                     the valid ones distinct in a row
+ *   teacher [B, nq, k] fp32 weights >= 0 aligned with idx's slots (any
+ *           scale: each row is renormalised over its valid slots)
+ *   grad_scale   dL/dKL_t of the caller's loss (1 for the plain sum of
+ *                eq. (8), 1/rows for a mean)
+ * Outputs (all fp32; every one but kl_out may be NULL to skip it):
+ *   kl_out          [B, nq]        KL_t (0 for a row with no valid slot or
+ *                                  a teacher with no mass on it)
+ *   grad_logits_out [B, nq, k]     dL/dI_{t,s} = grad_scale (softmax - p),
+ *                                  0 in unused slots
+ *   dq_out          [B, nq, HI, dI] dL/dq^I (overwritten)
+ *   dw_out          [B, nq, HI]     dL/dw   (overwritten)
+ *   dk_out          [B, kv_len, dI] dL/dk^I ADDED to the buffer (several
+ *                                  rows select the same key; the caller
+ *                                  zeroes it first), in an unspecified
+ *                                  order (float atomics)
+ * The ReLU of eq. (1) has derivative 0 at 0.  dq and dk are accumulated
+ * from bf16-rounded G = g * w * [q.k > 0] products in fp32.
+ * Supported: HI 1..64, dI in {32, 64, 128}, k <= 4096.  Pointers 16-byte
+ * aligned (dq, dk 8).  Indices outside [-1, kv_len) are skipped and set
+ * DSA_ERR_DEVICE_CHECK (detail 0xA77E) in the workspace status.
+ * ---------------------------------------------------------------------- */
+size_t dsa_indexer_kl_workspace(void);
+dsa_status dsa_indexer_kl_sparse(int B, int nq, int kv_len, int HI, int dI, int k, const void* qI, const void* kI,
+                                 const float* w, const int32_t* idx, const float* teacher, float grad_scale,
+                                 float* kl_out, float* grad_logits_out, float* dq_out, float* dw_out, float* dk_out,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

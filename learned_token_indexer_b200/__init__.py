@@ -243,6 +243,44 @@ def selection_overlap(idx_teacher, idx_student, max_pos: int, return_counts: boo
 
 
 # --------------------------------------------------------------------------
+# Training: sparse-stage indexer KL (eq. (8))
+# --------------------------------------------------------------------------
+
+def indexer_kl_sparse(qI, kI, w, idx, teacher, grad_scale: float = 1.0, grads=("dq", "dw", "dk"),
+                      grad_logits: bool = False, dk_out=None, workspace: Optional[Workspace] = None):
+    """KL_t of eq. (8) on each row's selected set, with the gradients of a
+    loss L (dL/dKL_t = grad_scale) with respect to qI, w and kI.
+
+    qI [B, nq, HI, dI] bf16, kI [B, kv_len, dI] bf16, w [B, nq, HI] fp32,
+    idx [B, nq, k] int32, teacher [B, nq, k] fp32 (renormalised per row over
+    the valid slots).  Returns a dict with "kl" [B, nq] and the requested
+    gradients (fp32): "dq", "dw", "dk" [B, kv_len, dI] (added to dk_out when
+    given, else to a fresh zero buffer) and "grad_logits" [B, nq, k]."""
+    B, nq, HI, dI = qI.shape
+    kv_len = kI.shape[1]
+    k = idx.shape[-1]
+    dev = qI.device
+    if qI.dtype != torch.bfloat16 or kI.dtype != torch.bfloat16:
+        raise TypeError("the KL path takes bfloat16 indexer operands")
+    out = {"kl": torch.empty((B, nq), dtype=torch.float32, device=dev)}
+    if "dq" in grads:
+        out["dq"] = torch.empty((B, nq, HI, dI), dtype=torch.float32, device=dev)
+    if "dw" in grads:
+        out["dw"] = torch.empty((B, nq, HI), dtype=torch.float32, device=dev)
+    if "dk" in grads:
+        out["dk"] = dk_out if dk_out is not None else torch.zeros((B, kv_len, dI), dtype=torch.float32, device=dev)
+    if grad_logits:
+        out["grad_logits"] = torch.empty((B, nq, k), dtype=torch.float32, device=dev)
+    L = lib()
+    wsb = _ws(workspace, dev).get(L.dsa_indexer_kl_workspace())
+    _check(L.dsa_indexer_kl_sparse(B, nq, kv_len, HI, dI, k, _ptr(qI), _ptr(kI), _ptr(w), _ptr(idx), _ptr(teacher),
+                                   float(grad_scale), _ptr(out["kl"]), _ptr(out.get("grad_logits")),
+                                   _ptr(out.get("dq")), _ptr(out.get("dw")), _ptr(out.get("dk")), _ptr(wsb),
+                                   wsb.numel(), _stream(dev)))
+    return out
+
+
+# --------------------------------------------------------------------------
 # Debug / test
 # --------------------------------------------------------------------------
 

@@ -478,4 +478,48 @@ dsa_status dsa_selection_overlap(int rows, int k, int max_pos, const int32_t* id
   return DSA_OK;
 }
 
+// ---------------------------------------------------------------- training: indexer KL (eq. 8)
+size_t dsa_indexer_kl_workspace(void) { return kHeader; }
+
+dsa_status dsa_indexer_kl_sparse(int B, int nq, int kv_len, int HI, int dI, int k, const void* qI, const void* kI,
+                                 const float* w, const int32_t* idx, const float* teacher, float grad_scale,
+                                 float* kl_out, float* grad_logits_out, float* dq_out, float* dw_out, float* dk_out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  DSA_CHECK(B >= 1 && nq >= 0 && kv_len >= 1 && k >= 1, DSA_ERR_INVALID_ARG,
+            "need B >= 1, nq >= 0, kv_len >= 1, k >= 1");
+  DSA_CHECK(HI >= 1 && HI <= 64, DSA_ERR_UNSUPPORTED, "HI=%d: the KL kernel supports 1..64 indexer heads", HI);
+  DSA_CHECK(dI == 32 || dI == 64 || dI == 128, DSA_ERR_UNSUPPORTED, "dI=%d: supported are 32, 64, 128", dI);
+  DSA_CHECK(k <= dsa::kMaxKLTopk, DSA_ERR_UNSUPPORTED, "k=%d above %d (the row's scores live in shared memory)", k,
+            dsa::kMaxKLTopk);
+  DSA_CHECK((int64_t)B * nq <= INT32_MAX, DSA_ERR_UNSUPPORTED, "too many rows");
+  DSA_CHECK(qI && kI && w && idx && teacher && kl_out, DSA_ERR_INVALID_ARG, "null tensor pointer");
+  DSA_CHECK(aligned(qI, 16) && aligned(kI, 16), DSA_ERR_INVALID_ARG, "qI and kI must be 16-byte aligned");
+  DSA_CHECK((!dq_out || aligned(dq_out, 8)) && (!dk_out || aligned(dk_out, 8)), DSA_ERR_INVALID_ARG,
+            "dq and dk must be 8-byte aligned");
+  DSA_CHECK(std::isfinite(grad_scale), DSA_ERR_INVALID_ARG, "grad_scale must be finite");
+  if (dsa_status st = check_ws(workspace, workspace_bytes, kHeader)) return st;
+  if (nq == 0) return DSA_OK;
+  dsa::KLArgs a{};
+  a.rows = B * nq;
+  a.nq = nq;
+  a.kv_len = kv_len;
+  a.HI = HI;
+  a.k = k;
+  a.grad_scale = grad_scale;
+  a.q = static_cast<const uint16_t*>(qI);
+  a.kI = static_cast<const uint16_t*>(kI);
+  a.w = w;
+  a.idx = idx;
+  a.teacher = teacher;
+  a.kl = kl_out;
+  a.grad_logits = grad_logits_out;
+  a.dq = dq_out;
+  a.dw = dw_out;
+  a.dk = dk_out;
+  a.status = status_of(workspace);
+  cudaError_t e = dsa::launch_indexer_kl(dI, a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "indexer_kl launch");
+  return DSA_OK;
+}
+
 }  // extern "C"

@@ -78,6 +78,24 @@ struct AttnArgs {
   DeviceStatus* status;
 };
 
+// Sparse-stage indexer KL on the selected set, forward and backward (indexer_kl.cu).
+constexpr int kMaxKLTopk = 4096;
+struct KLArgs {
+  int rows, nq, kv_len, HI, k;
+  float grad_scale;            // dL/dKL_t for every row
+  const uint16_t* q;           // [rows, HI, dI] bf16
+  const uint16_t* kI;          // [B, kv_len, dI] bf16
+  const float* w;              // [rows, HI]
+  const int32_t* idx;          // [rows, k]
+  const float* teacher;        // [rows, k]
+  float* kl;                   // [rows]
+  float* grad_logits;          // [rows, k] or null
+  float* dq;                   // [rows, HI, dI] or null
+  float* dw;                   // [rows, HI] or null
+  float* dk;                   // [B, kv_len, dI] (accumulated) or null
+  DeviceStatus* status;
+};
+
 cudaError_t launch_indexer_scan(int HI, bool fp8, int kblocks, const CUtensorMap& tq, const CUtensorMap& tk,
                                 const ScanArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_indexer_topk_prefill(int HI, bool fp8, int kblocks, const CUtensorMap& tq,
@@ -88,6 +106,8 @@ cudaError_t launch_fill_trivial_rows(int B, int nq, int q_offset, int rows_per_s
                                      cudaStream_t stream);
 cudaError_t launch_fill_f32(float* p, int64_t n, float v, cudaStream_t stream);
 cudaError_t launch_sparse_attn(const AttnArgs& a, int grid, cudaStream_t stream);
+size_t indexer_kl_smem_bytes(int dI, int k);
+cudaError_t launch_indexer_kl(int dI, const KLArgs& a, cudaStream_t stream);
 cudaError_t launch_wait_selftest(DeviceStatus* status, uint64_t timeout_ns, cudaStream_t stream);
 cudaError_t launch_selection_overlap(int rows, int k, int max_pos, const int32_t* idx_a, const int32_t* idx_b,
                                      int32_t* inter, int32_t* count_a, int grid, cudaStream_t stream);

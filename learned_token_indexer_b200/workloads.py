@@ -190,3 +190,41 @@ def sample_rows(w: Workload, nrows: int = 256, n: Optional[int] = None, salt: in
         i = int(torch.randint(0, n, (1,), generator=g))
         rows.add((b, i))
     return sorted(rows)
+
+
+def make_selection(B: int, nq: int, kv_len: int, k: int, q_offset: int = 0, seed: int = 0,
+                   device="cpu", rows_per_draw: int = 2048) -> torch.Tensor:
+    """Seeded synthetic selections (input of the sparse-stage KL, not a top-k).
+
+    Row i of each sequence sits at t = q_offset + i and holds min(k, t + 1)
+    distinct positions drawn uniformly from [0, t] in random slot order,
+    then -1 in the unused slots.  Returns int32 [B, nq, k] on ``device``.
+    """
+    g = _gen(device, seed + 77)
+    out = torch.empty((B, nq, k), dtype=torch.int32, device=device)
+    pos = torch.arange(kv_len, device=device)
+    for b in range(B):
+        for r0 in range(0, nq, rows_per_draw):
+            r1 = min(nq, r0 + rows_per_draw)
+            t = (q_offset + torch.arange(r0, r1, device=device))[:, None]
+            u = torch.rand((r1 - r0, kv_len), generator=g, device=device)
+            u = torch.where(pos[None, :] <= t, u, torch.full_like(u, 2.0))      # keys after t never drawn
+            kk = min(k, kv_len)
+            sel = torch.topk(u, kk, dim=1, largest=False).indices
+            sel = torch.where(sel <= t, sel, torch.full_like(sel, -1))
+            # valid first, then -1 (the index semantics of the prefill selector)
+            key = torch.where(sel >= 0, torch.zeros_like(sel), torch.ones_like(sel))
+            sel = torch.gather(sel, 1, torch.sort(key, dim=1, stable=True).indices)
+            row = torch.full((r1 - r0, k), -1, dtype=torch.int32, device=device)
+            row[:, :kk] = sel.to(torch.int32)
+            out[b, r0:r1] = row
+    return out
+
+
+def make_teacher(shape, seed: int = 0, device="cpu", zero_frac: float = 0.1) -> torch.Tensor:
+    """Seeded synthetic teacher weights >= 0 (fp32) with a fraction of exact
+    zeros; entries in unused slots are drawn too (the KL ignores them)."""
+    g = _gen(device, seed + 91)
+    t = torch.rand(shape, generator=g, device=device) ** 3
+    z = torch.rand(shape, generator=g, device=device) < zero_frac
+    return torch.where(z, torch.zeros_like(t), t).float().contiguous()

@@ -115,3 +115,22 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         _lib.load()
+
+
+def test_indexer_kl_argument_checks(lib):
+    f = lib.dsa_indexer_kl_sparse
+    v = C.c_void_p(256)
+
+    def call(B=1, nq=4, kv_len=16, HI=64, dI=128, k=8, q=v, grad_scale=1.0, ws=v, wsb=256):
+        return f(B, nq, kv_len, HI, dI, k, q, v, v, v, v, grad_scale, v, None, None, None, None, ws, wsb, None)
+
+    assert call(HI=65) == 2                      # more heads than the kernel pads to
+    assert call(dI=48) == 2
+    assert call(k=4097) == 2                     # the row's scores live in shared memory
+    assert call(k=0) == 1
+    assert call(q=None) == 1
+    assert call(q=C.c_void_p(264)) == 1          # misaligned operand
+    assert call(grad_scale=float("inf")) == 1
+    assert call(wsb=8) == 3
+    assert call(nq=0) == 0                       # nothing to do
+    assert lib.dsa_indexer_kl_workspace() == 256
