@@ -8,7 +8,10 @@ the fused Lightning Indexer + causal top-k (eqs. (1)-(2) of the page
 rows (eq. (3)).  The default workload is the integer-valued prefill
 (B=1, n=8192, HI=64, dI=128, k=2048, 16 heads, latent 576/512); the metric is
 query tokens per second.  --workload decode|prefill_fp8|long_prefill|tiny
-selects the other workloads.
+selects the other workloads; --workload indexer_kl times the sparse training
+stage's indexer step instead: selection, the sparse attention forward with
+its lse, the teacher recomputed on the selected set, then the eq. (8) KL on
+that set, forward and backward.
 
 Timing: W warm-up steps, then exactly K steps, each bracketed by CUDA events
 on the launching stream; L2 is flushed (a 256 MiB write) before every timed
@@ -45,6 +48,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 METRIC = {
     "prefill": ("prefill query-tokens/s (indexer+top-k+sparse attn)", "query-tokens/s"),
     "decode": ("decode tokens/s (indexer scan+top-k+sparse attn)", "tokens/s"),
+    "train": ("sparse-stage indexer training query-tokens/s (indexer+top-k, sparse attn, teacher, eq. 8 KL fwd/bwd)",
+              "query-tokens/s"),
 }
 
 
@@ -186,22 +191,25 @@ class PrefillRun:
             kw = dict(self.kw)
             if w.fp8 and self.chunk != w.n:
                 kw["q_scale"] = self.kw["q_scale"][sl].contiguous()
-            if ev is not None:
-                ev["idx"][0].append(self._rec())
+            e0 = self._rec(ev)
             dsa.indexer_topk_prefill(d["qI"][sl], d["kI"], d["w"][sl], w.k, q_offset=c0, idx_out=self.idx[sl],
                                      workspace=self.ws_idx, **kw)
-            if ev is not None:
-                ev["idx"][1].append(self._rec())
+            e1 = self._rec(ev)
             dsa.sparse_attn_prefill(d["q"][sl], d["latent"], self.idx[sl], w.Dv, scale=w.scale, out=self.out[sl],
                                     workspace=self.ws_att)
+            e2 = self._rec(ev)
             if ev is not None:
-                ev["attn"][1].append(self._rec())
+                ev["indexer_topk_prefill"].append((e0, e1))
+                ev["sparse_attn"].append((e1, e2))
             triv = c0 < w.k
             launches += 2 + (1 if triv else 0)
         self.launches_per_step = launches
 
     @staticmethod
-    def _rec():
+    def _rec(ev=True):
+        """A recorded timing event (None when the step is not being timed)."""
+        if ev is None:
+            return None
         e = torch.cuda.Event(enable_timing=True)
         e.record()
         return e
@@ -278,17 +286,17 @@ class DecodeRun:
 
     def step(self, ev=None):
         dsa, w, d = self.dsa, self.w, self.d
-        if ev is not None:
-            ev["idx"][0].append(PrefillRun._rec())
+        e0 = PrefillRun._rec(ev)
         dsa.indexer_topk_decode(d["qI"], d["w"], d["kI_cache"], d["cu_seqlens"], w.k, self.total, self.maxlen,
                                 q_scale=d.get("q_scale"), k_scale=d.get("k_scale"), idx_out=self.idx,
                                 workspace=self.ws_idx)
-        if ev is not None:
-            ev["idx"][1].append(PrefillRun._rec())
+        e1 = PrefillRun._rec(ev)
         dsa.sparse_attn_decode(d["q"], d["latent_cache"], d["cu_seqlens"], self.idx, w.Dv, self.total,
                                scale=w.scale, out=self.out, workspace=self.ws_att)
+        e2 = PrefillRun._rec(ev)
         if ev is not None:
-            ev["attn"][1].append(PrefillRun._rec())
+            ev["indexer_topk_decode"].append((e0, e1))
+            ev["sparse_attn_decode"].append((e1, e2))
 
     def rows(self):
         return self.w.B
@@ -323,9 +331,85 @@ class DecodeRun:
         return self.out
 
 
+class TrainRun(PrefillRun):
+    """Sparse training stage, indexer side (§1.2): the fused indexer + top-k
+    selects S_t; the sparse attention forward (eq. (3)) returns its lse; the
+    teacher is recomputed on S_t from it (heads summed, L1-normalised); then
+    the eq. (8) KL on S_t with dq, dw and dk (dk is zeroed inside the step:
+    it accumulates)."""
+
+    def __init__(self, w: W.Workload, device):
+        import learned_token_indexer_b200 as dsa
+        self.dsa, self.w, self.dev = dsa, w, device
+        self.d = W.make_prefill_inputs(w, device)
+        self.ws_idx = dsa.Workspace(device)
+        self.ws_att = dsa.Workspace(device)
+        self.idx = torch.empty((w.B, w.n, w.k), dtype=torch.int32, device=device)
+        self.out = torch.empty((w.B, w.n, w.H, w.Dv), dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty((w.B, w.n, w.H), dtype=torch.float32, device=device)
+        self.teacher = torch.empty((w.B, w.n, w.k), dtype=torch.float32, device=device)
+        self.dk = torch.zeros((w.B, w.n, w.dI), dtype=torch.float32, device=device)
+        self.res = None
+        self.launches_per_step = 0
+
+    def step(self, ev=None):
+        dsa, w, d = self.dsa, self.w, self.d
+        e0 = self._rec(ev)
+        dsa.indexer_topk_prefill(d["qI"], d["kI"], d["w"], w.k, idx_out=self.idx, workspace=self.ws_idx)
+        e1 = self._rec(ev)
+        dsa.sparse_attn_prefill(d["q"], d["latent"], self.idx, w.Dv, scale=w.scale, out=self.out, lse=self.lse,
+                                workspace=self.ws_att)
+        e2 = self._rec(ev)
+        dsa.attn_teacher_prefill(d["q"], d["latent"], self.idx, self.lse, scale=w.scale, out=self.teacher,
+                                 workspace=self.ws_att)
+        e3 = self._rec(ev)
+        self.dk.zero_()
+        self.res = dsa.indexer_kl_sparse(d["qI"], d["kI"], d["w"], self.idx, self.teacher, grad_scale=1.0 / w.n,
+                                         dk_out=self.dk, workspace=self.ws_att)
+        e4 = self._rec(ev)
+        if ev is not None:
+            for name, a, b in (("indexer_topk_prefill", e0, e1), ("sparse_attn", e1, e2), ("attn_teacher", e2, e3),
+                               ("indexer_kl", e3, e4)):
+                ev[name].append((a, b))
+        # fill_trivial_rows, indexer_topk_prefill, sparse_attn, attn_teacher, indexer_kl
+        self.launches_per_step = 5
+
+    def selection_diagnostics(self):
+        return None
+
+    def kernel_work(self):
+        w = self.w
+        pairs = count_pairs_needed(0, w.n, w.k)
+        ent = selected_entries(0, w.n, w.k)
+        return {
+            "indexer_topk_prefill": {"flops": 2 * w.HI * w.dI * w.B * pairs, "unit": "TFLOP/s",
+                                     "per_unit": f"2*HI*dI = {2 * w.HI * w.dI} FLOP per scored (t,s) pair",
+                                     "units": w.B * pairs},
+            "sparse_attn": {"flops": 2 * w.H * w.B * ent * (w.Dqk + w.Dv), "unit": "TFLOP/s",
+                            "per_unit": f"2*H*(Dqk+Dv) = {2 * w.H * (w.Dqk + w.Dv)} FLOP per selected entry",
+                            "units": w.B * ent},
+            "attn_teacher": {"flops": 2 * w.H * w.B * ent * w.Dqk, "unit": "TFLOP/s",
+                             "per_unit": f"2*H*Dqk = {2 * w.H * w.Dqk} FLOP per selected entry (logits recompute)",
+                             "units": w.B * ent},
+            "indexer_kl": {"flops": 6 * w.HI * w.dI * w.B * ent, "unit": "TFLOP/s",
+                           "per_unit": (f"6*HI*dI = {6 * w.HI * w.dI} FLOP per selected entry (scores, dq, dk: "
+                                        "three HI x dI products; the kernel's recompute is not counted)"),
+                           "units": w.B * ent},
+        }
+
+    def host_inputs(self):
+        return {k: self.d[k].cpu().pin_memory() for k in ("qI", "kI", "w", "q", "latent")}
+
+    def result(self):
+        if self.res is None:
+            self.step()
+        return self.res["kl"]
+
+
 def time_steps(run, steps, flush):
-    """Per-step and per-kernel device times (ms) over `steps` timed steps."""
-    ev = {"idx": ([], []), "attn": ([], [])}
+    """Per-step device times (ms) and, per kernel, the duration of each
+    launch (ms) over `steps` timed steps."""
+    ev = {name: [] for name in run.kernel_work()}
     starts, ends = [], []
     for _ in range(steps):
         flush.fill_(1)
@@ -336,10 +420,8 @@ def time_steps(run, steps, flush):
         ends.append(e)
     torch.cuda.synchronize()
     step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
-    idx_ms = [a.elapsed_time(b) for a, b in zip(*ev["idx"])]
-    # attention segments start where the indexer segment of the same chunk ends
-    attn_ms = [a.elapsed_time(b) for a, b in zip(ev["idx"][1], ev["attn"][1])]
-    return step_ms, idx_ms, attn_ms
+    seg_ms = {name: [a.elapsed_time(b) for a, b in pairs] for name, pairs in ev.items()}
+    return step_ms, seg_ms
 
 
 def time_e2e(run, steps):
@@ -385,21 +467,43 @@ def cpu_baseline(w: W.Workload, budget_s: float = 15.0, run_inputs=None):
         dt = time.perf_counter() - t0
         return {"value": done / dt, "unit": METRIC["decode"][1], "cores": threads, "kind": "oracle",
                 "sample": f"{done} of {w.B} sequences of one decode step (float64 numpy)"}
-    d = run_inputs if run_inputs is not None else W.make_prefill_inputs(w, "cpu")
+    d = run_inputs if run_inputs is not None else _host_prefill_inputs(w)
     rows = W.sample_rows(w, 4096)
     rng = np.random.default_rng(7)
     rng.shuffle(rows)
+    one = _oracle_train_row if w.kind == "train" else _oracle_row
     t0 = time.perf_counter()
     done = 0
     for b, i in rows:
-        _oracle_row(O, w, d, b, i)
+        one(O, w, d, b, i)
         done += 1
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    return {"value": done / dt, "unit": METRIC["prefill"][1], "cores": threads, "kind": "oracle",
-            "sample": f"{done} seeded query rows of B*n={w.B * w.n} (uniform over positions), indexer + top-k + "
-                      f"attention per row, float64 numpy"}
+    what = ("indexer + top-k + attention + teacher + eq. (8) KL with gradients" if w.kind == "train"
+            else "indexer + top-k + attention")
+    return {"value": done / dt, "unit": METRIC[w.kind][1], "cores": threads, "kind": "oracle",
+            "sample": f"{done} seeded query rows of B*n={w.B * w.n} (uniform over positions), {what} per row, "
+                      f"float64 numpy"}
+
+
+def _host_prefill_inputs(w):
+    return W.make_prefill_inputs(w, "cpu")
+
+
+def _oracle_train_row(O, w, d, b, i):
+    """One row of the sparse-stage indexer step: selection, attention forward,
+    teacher on S_t, eq. (8) KL with gradients."""
+    q = d["qI"][b, i].double().numpy()
+    kk = d["kI"][b].double().numpy()
+    ww = d["w"][b, i].double().numpy()
+    s = O.indexer_scores_row(q, kk[: i + 1], ww)
+    sel = O.causal_topk_row(s, i, w.k)
+    qa = d["q"][b, i].double().numpy()
+    lat = d["latent"][b].double().numpy()
+    O.sparse_attention_row(qa, lat, sel, w.scale, w.Dv)
+    p = O.attention_teacher_row(qa, lat, sel, w.scale)
+    O.indexer_kl_sparse_row(q, kk, ww, sel, p, 1.0 / w.n)
 
 
 def _oracle_row(O, w, d, b, i):
@@ -441,6 +545,9 @@ def workload_label(w: W.Workload):
                 f"{'fp8-e4m3' if w.fp8 else 'bf16'} K^I cache; "
                 f"attn H={w.H} latent {w.Dqk}/{w.Dv}")
     dt = "fp8-e4m3 indexer" if w.fp8 else ("bf16 integer-valued indexer" if w.integer_valued else "bf16 indexer")
+    if w.kind == "train":
+        return (f"sparse-stage indexer step: prefill B={w.B} n={w.n} HI={w.HI} dI={w.dI} k={w.k} {dt}; "
+                f"attn H={w.H} latent {w.Dqk}/{w.Dv} with lse; teacher on S_t from it; KL fwd + dq, dw, dk")
     ch = f" in {w.chunk}-query chunks" if w.chunk else ""
     return (f"prefill B={w.B} n={w.n} HI={w.HI} dI={w.dI} k={w.k} {dt}{ch}; attn H={w.H} latent {w.Dqk}/{w.Dv}")
 
@@ -483,7 +590,7 @@ def run_b200(args):
     if world > 1:
         torch.distributed.barrier()
     w = rank_workload(W.ALL[args.workload], rank)
-    run = DecodeRun(w, dev) if w.kind == "decode" else PrefillRun(w, dev)
+    run = {"decode": DecodeRun, "train": TrainRun}.get(w.kind, PrefillRun)(w, dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         run.step()
@@ -495,7 +602,7 @@ def run_b200(args):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    step_ms, idx_ms, attn_ms = time_steps(run, args.steps, flush)
+    step_ms, seg_ms = time_steps(run, args.steps, flush)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -507,7 +614,7 @@ def run_b200(args):
     if not args.no_e2e:
         e2e_ms, h2d, d2h = time_e2e(run, max(3, min(10, args.steps)))
         e2e_ms = max_over_ranks(e2e_ms, dev)
-        e2e = {"value": job_throughput(world, run.rows(), e2e_ms), "unit": METRIC[w.kind if w.kind == "decode" else "prefill"][1],
+        e2e = {"value": job_throughput(world, run.rows(), e2e_ms), "unit": METRIC[w.kind][1],
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
     if world > 1:
         torch.distributed.barrier()
@@ -517,13 +624,11 @@ def run_b200(args):
     peaks, peak_src = load_peaks()
     work = run.kernel_work()
     names = list(work.keys())
-    kms = {names[0]: float(np.mean(idx_ms)) / max(1, len(idx_ms) // max(1, args.steps)),
-           names[1]: float(np.mean(attn_ms)) / max(1, len(attn_ms) // max(1, args.steps))}
-    # per launch: each step launches each kernel once per chunk
-    per_step_launches = max(1, len(idx_ms) // max(1, args.steps))
     kernels = {}
     for name, wk in work.items():
-        t_launch = float(np.mean(idx_ms if name == names[0] else attn_ms))
+        # per launch: each step launches each kernel once per chunk
+        per_step_launches = max(1, len(seg_ms[name]) // max(1, args.steps))
+        t_launch = float(np.mean(seg_ms[name]))
         if "flops" in wk:
             per_launch = wk["flops"] / per_step_launches
             peak = peaks["bf16_tflops"] * (2.0 if (w.fp8 and name == names[0]) else 1.0)
@@ -543,7 +648,7 @@ def run_b200(args):
     roof = {k: kernels[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roof["kernel"] = dom
     roof["peak_source"] = f"{peak_src} ({'fp8 = 2 x measured bf16' if (w.fp8 and roof['bound'] == 'tensor' and dom == names[0]) else 'burst bf16 / copy bandwidth'})"
-    metric, unit = METRIC["decode" if w.kind == "decode" else "prefill"]
+    metric, unit = METRIC[w.kind]
     line = {
         "metric": metric, "value": job_throughput(world, run.rows(), ms), "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -579,7 +684,7 @@ def run_reference(args):
         return
     import oracle as O
     w = W.ALL[args.workload]
-    metric, unit = METRIC["decode" if w.kind == "decode" else "prefill"]
+    metric, unit = METRIC[w.kind]
     total_budget = args.ref_budget
     nsteps = args.steps + args.warmup
     if w.kind == "decode":
@@ -595,11 +700,12 @@ def run_reference(args):
         units = list(range(w.B))
         unit_name = "sequences"
     else:
-        d = W.make_prefill_inputs(w, "cpu")
+        d = _host_prefill_inputs(w)
         units = W.sample_rows(w, 4096)
         np.random.default_rng(7).shuffle(units)
+        row_fn = _oracle_train_row if w.kind == "train" else _oracle_row
         def one(u):
-            _oracle_row(O, w, d, *u)
+            row_fn(O, w, d, *u)
         unit_name = "query rows"
     t0 = time.perf_counter()
     one(units[0])

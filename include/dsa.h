@@ -75,9 +75,10 @@ dsa_status dsa_workspace_init(void* workspace, size_t workspace_bytes, void* str
  * (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_CHECK), store its detail word in
  * *detail if non-NULL, and clear it.  The first failure of a launch wins.
  * Detail words: DSA_ERR_TIMEOUT -> the wait that gave up (0x1xxx indexer
- * prefill, 0x2xxx sparse attention, 0x1xx..0x3xx indexer scan, 0x7e57
- * self-test);
- * DSA_ERR_DEVICE_CHECK -> 0xA77E an attention index outside [-1, L),
+ * prefill, 0x2xxx sparse attention, 0x3101 sparse-stage teacher,
+ * 0x1xx..0x3xx indexer scan, 0x7e57 self-test);
+ * DSA_ERR_DEVICE_CHECK -> 0xA77E an attention, teacher or KL index outside
+ * [-1, L),
  * 0x70E1 a top-k row longer than its matrix, 0x5e1ec6..0x5e1ec9 a selection
  * whose candidate count broke its invariant (output slots may then hold
  * any in-range position or -1). */
@@ -247,7 +248,7 @@ dsa_status dsa_selection_overlap(int rows, int k, int max_pos, const int32_t* id
  * The ReLU of eq. (1) has derivative 0 at 0.  dq and dk are accumulated
  * from bf16-rounded G = g * w * [q.k > 0] products in fp32.
  * Supported: HI 1..64, dI in {32, 64, 128}, k <= 4096.  Pointers 16-byte
- * aligned (dq, dk 8).  Indices outside [-1, kv_len) are skipped and set
+ * aligned (dq 8).  Indices outside [-1, kv_len) are skipped and set
  * DSA_ERR_DEVICE_CHECK (detail 0xA77E) in the workspace status.
  * ---------------------------------------------------------------------- */
 size_t dsa_indexer_kl_workspace(void);
@@ -255,6 +256,27 @@ dsa_status dsa_indexer_kl_sparse(int B, int nq, int kv_len, int HI, int dI, int 
                                  const float* w, const int32_t* idx, const float* teacher, float grad_scale,
                                  float* kl_out, float* grad_logits_out, float* dq_out, float* dw_out, float* dk_out,
                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Sparse-stage teacher (§1.2, the remark after eq. (8), and eq. (16)).
+ * When the teacher of eq. (8) comes from the current sparse main attention
+ * it is already a distribution over S_t: the heads' attention probabilities
+ * a_h(s) = exp(scale q_{t,h} . c_s - lse_{t,h}) summed over the heads and
+ * L1-normalised along the selected positions (the DSA aggregation).  This
+ * recomputes the attention scores of the selected set from the forward's
+ * lse; nothing else of the forward is kept.
+ *   q [B, nq, H, Dqk] bf16, latent [B, kv_len, Dqk] bf16, idx [B, nq, k]
+ *   (as given to dsa_sparse_attn_prefill), lse [B, nq, H] fp32 (its lse
+ *   output), scale (its scale).
+ *   p_out [B, nq, k] fp32: p_{t,s} per slot, 0 in unused slots; a row
+ *   with no valid slot is all 0.
+ * Supported: Dqk a multiple of 16 up to 576, k <= 4096, any H.  q and latent
+ * 16-byte aligned.  Indices outside [-1, kv_len) are skipped and set
+ * DSA_ERR_DEVICE_CHECK (detail 0xA77E).
+ * ---------------------------------------------------------------------- */
+dsa_status dsa_attn_teacher_prefill(int B, int nq, int kv_len, int H, int Dqk, int k, float scale, const void* q,
+                                    const void* latent, const int32_t* idx, const float* lse, float* p_out,
+                                    void* workspace, size_t workspace_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -16,6 +16,7 @@ Entry points (page "2.2.1 · DSA 与索引器", §1.1 eqs. (1)-(3), §2 decode):
 from __future__ import annotations
 
 import ctypes as C
+import math
 from typing import Optional
 
 import torch
@@ -277,6 +278,28 @@ def indexer_kl_sparse(qI, kI, w, idx, teacher, grad_scale: float = 1.0, grads=("
                                    float(grad_scale), _ptr(out["kl"]), _ptr(out.get("grad_logits")),
                                    _ptr(out.get("dq")), _ptr(out.get("dw")), _ptr(out.get("dk")), _ptr(wsb),
                                    wsb.numel(), _stream(dev)))
+    return out
+
+
+def attn_teacher_prefill(q, latent, idx, lse, scale: Optional[float] = None, out=None,
+                         workspace: Optional[Workspace] = None):
+    """Teacher of eq. (8) from the sparse attention: per slot of idx, the
+    heads' attention probabilities (recomputed with the forward's lse)
+    summed over heads and L1-normalised over the row's selected positions.
+    q [B, nq, H, Dqk] bf16, latent [B, kv_len, Dqk] bf16, idx [B, nq, k],
+    lse [B, nq, H] fp32 (from sparse_attn_prefill).  Returns [B, nq, k] fp32."""
+    B, nq, H, Dqk = q.shape
+    kv_len = latent.shape[1]
+    k = idx.shape[-1]
+    dev = q.device
+    if scale is None:
+        scale = 1.0 / math.sqrt(Dqk)
+    if out is None:
+        out = torch.empty((B, nq, k), dtype=torch.float32, device=dev)
+    L = lib()
+    wsb = _ws(workspace, dev).get(L.dsa_small_workspace())
+    _check(L.dsa_attn_teacher_prefill(B, nq, kv_len, H, Dqk, k, float(scale), _ptr(q), _ptr(latent), _ptr(idx),
+                                      _ptr(lse), _ptr(out), _ptr(wsb), wsb.numel(), _stream(dev)))
     return out
 
 

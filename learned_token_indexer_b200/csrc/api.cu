@@ -494,8 +494,8 @@ dsa_status dsa_indexer_kl_sparse(int B, int nq, int kv_len, int HI, int dI, int 
   DSA_CHECK((int64_t)B * nq <= INT32_MAX, DSA_ERR_UNSUPPORTED, "too many rows");
   DSA_CHECK(qI && kI && w && idx && teacher && kl_out, DSA_ERR_INVALID_ARG, "null tensor pointer");
   DSA_CHECK(aligned(qI, 16) && aligned(kI, 16), DSA_ERR_INVALID_ARG, "qI and kI must be 16-byte aligned");
-  DSA_CHECK((!dq_out || aligned(dq_out, 8)) && (!dk_out || aligned(dk_out, 8)), DSA_ERR_INVALID_ARG,
-            "dq and dk must be 8-byte aligned");
+  DSA_CHECK((!dq_out || aligned(dq_out, 8)) && (!dk_out || aligned(dk_out, 16)), DSA_ERR_INVALID_ARG,
+            "dq must be 8-byte and dk 16-byte aligned");
   DSA_CHECK(std::isfinite(grad_scale), DSA_ERR_INVALID_ARG, "grad_scale must be finite");
   if (dsa_status st = check_ws(workspace, workspace_bytes, kHeader)) return st;
   if (nq == 0) return DSA_OK;
@@ -519,6 +519,40 @@ dsa_status dsa_indexer_kl_sparse(int B, int nq, int kv_len, int HI, int dI, int 
   a.status = status_of(workspace);
   cudaError_t e = dsa::launch_indexer_kl(dI, a, (cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "indexer_kl launch");
+  return DSA_OK;
+}
+
+dsa_status dsa_attn_teacher_prefill(int B, int nq, int kv_len, int H, int Dqk, int k, float scale, const void* q,
+                                    const void* latent, const int32_t* idx, const float* lse, float* p_out,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  DSA_CHECK(B >= 1 && nq >= 0 && kv_len >= 1 && k >= 1 && H >= 1, DSA_ERR_INVALID_ARG,
+            "need B >= 1, nq >= 0, kv_len >= 1, k >= 1, H >= 1");
+  DSA_CHECK(Dqk >= 16 && Dqk <= 576 && Dqk % 16 == 0, DSA_ERR_UNSUPPORTED,
+            "Dqk=%d: supported are multiples of 16 up to 576", Dqk);
+  DSA_CHECK(k <= dsa::kMaxTeacherTopk, DSA_ERR_UNSUPPORTED, "k=%d above %d", k, dsa::kMaxTeacherTopk);
+  DSA_CHECK((int64_t)B * nq <= INT32_MAX, DSA_ERR_UNSUPPORTED, "too many rows");
+  DSA_CHECK(q && latent && idx && lse && p_out, DSA_ERR_INVALID_ARG, "null tensor pointer");
+  DSA_CHECK(aligned(q, 16) && aligned(latent, 16), DSA_ERR_INVALID_ARG, "q and latent must be 16-byte aligned");
+  DSA_CHECK(std::isfinite(scale), DSA_ERR_INVALID_ARG, "scale must be finite");
+  if (dsa_status st = check_ws(workspace, workspace_bytes, kHeader)) return st;
+  if (nq == 0) return DSA_OK;
+  dsa::TeacherArgs a{};
+  a.rows = B * nq;
+  a.nq = nq;
+  a.kv_len = kv_len;
+  a.H = H;
+  a.Dqk = Dqk;
+  a.k = k;
+  a.scale = scale;
+  a.q = static_cast<const uint16_t*>(q);
+  a.latent = static_cast<const uint16_t*>(latent);
+  a.idx = idx;
+  a.lse = lse;
+  a.p_out = p_out;
+  a.status = status_of(workspace);
+  a.timeout_ns = dsa::wait_timeout_ns();
+  cudaError_t e = dsa::launch_attn_teacher(a, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "attn_teacher launch");
   return DSA_OK;
 }
 

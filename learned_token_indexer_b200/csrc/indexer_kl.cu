@@ -17,8 +17,8 @@
 //
 // One CTA (4 warps) per query row.  The row's queries stay in shared memory;
 // the selected key rows are gathered 64 at a time with 16-byte cp.async into
-// two stages of padded rows (zero-filled for unused slots).  Two passes over
-// the selected keys:
+// three stages of padded rows (zero-filled for unused slots), two chunks
+// ahead of the one being computed.  Two passes over the selected keys:
 //   pass 1: D = K_S Q^T on mma.sync (warp w owns keys 16w..16w+15 of a chunk,
 //           all heads), I_s = sum_j w_j ReLU(D_sj) -> shared memory;
 //   row:    softmax over S_t, teacher renormalisation, KL_t, g_s;
@@ -26,7 +26,8 @@
 //           G_sj = g_s w_j [D_sj > 0] is the A operand of dk = G Q (taken
 //           straight from the D accumulators) and, through shared memory,
 //           of dq = G^T K_S (warp w owns heads 16w..16w+15).  dk rows are
-//           added to global memory with float2 atomics.
+//           added to global memory with float4 atomics (lane pairs swap
+//           halves of their accumulator fragments to form 4 columns).
 // Chunks whose slots are all unused are skipped, so short rows (t < k) cost
 // what they select.  The heads are padded to 64 with zero queries and zero
 // weights (exact: their D, ReLU and G are 0).
@@ -42,6 +43,7 @@ namespace {
 constexpr int kChunk = 64;       // selected keys per chunk
 constexpr int kHP = 64;          // heads, padded
 constexpr int kThreads = 128;
+constexpr int kStages = 3;       // key-chunk stages in flight (two prefetched)
 constexpr int kMaxChunks = kMaxKLTopk / kChunk;
 
 template <int DI>
@@ -54,12 +56,12 @@ struct KLGeom {
   static constexpr int kQBytes = kHP * kPitch;
   static constexpr int kGPitch = kHP * 2 + 16;     // G rows (64 heads, bf16)
   static constexpr int kGBytes = kChunk * kGPitch;
-  // shared memory: Q | 2 K stages | G | w | positions | dw partials | scratch | chunk list | I / g
+  // shared memory: Q | K stages | G | w | positions | dw partials | scratch | chunk list | I / g
   static constexpr int kOffK = kQBytes;
-  static constexpr int kOffG = kOffK + 2 * kStageBytes;
+  static constexpr int kOffG = kOffK + kStages * kStageBytes;
   static constexpr int kOffW = kOffG + kGBytes;
   static constexpr int kOffPos = kOffW + kHP * 4;
-  static constexpr int kOffDw = kOffPos + 2 * kChunk * 4;
+  static constexpr int kOffDw = kOffPos + kStages * kChunk * 4;
   static constexpr int kOffRed = kOffDw + 4 * kHP * 4;
   static constexpr int kOffList = kOffRed + 16 * 4;
   static constexpr int kOffI = kOffList + (kMaxChunks + 4) * 4;
@@ -219,10 +221,10 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_kl_kernel(const KLArgs a)
     wr[nt][1] = sW[8 * nt + 2 * c + 1];
   }
 
-  // Gather the selected key rows of chunk list[v % nl] into stage v & 1.
+  // Gather the selected key rows of chunk list[v % nl] into stage v % kStages.
   auto load_chunk = [&](int v) {
     const int ch = list[v % nl];
-    const int st = v & 1;
+    const int st = v % kStages;
     const uint32_t dst0 = sk + st * G::kStageBytes;
     for (int p = tid; p < kChunk * G::kPieces; p += kThreads) {
       const int r = p / G::kPieces, pc = p % G::kPieces;
@@ -279,14 +281,19 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_kl_kernel(const KLArgs a)
   };
 
   const int V = backward ? 2 * nl : nl;
-  if (nl > 0) load_chunk(0);
+  if (V > 0) load_chunk(0);
+  cp_async_commit();
+  if (V > 1) load_chunk(1);
   cp_async_commit();
   for (int v = 0; v < V; ++v) {
-    if (v + 1 < V) load_chunk(v + 1);
-    cp_async_commit();
+    // Chunk v has landed once at most one newer group is pending; after the
+    // barrier every thread is done with chunk v - 1, whose stage the load of
+    // chunk v + 2 reuses.
     cp_async_wait<1>();
     __syncthreads();
-    const int st = v & 1;
+    if (v + 2 < V) load_chunk(v + 2);
+    cp_async_commit();
+    const int st = v % kStages;
     const int ch = list[v % nl];
     const uint32_t stage = sk + st * G::kStageBytes;
     const int slot0 = ch * kChunk + 16 * warp + g, slot1 = slot0 + 8;
@@ -327,10 +334,10 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_kl_kernel(const KLArgs a)
         st_shared_u32(sg + (16 * warp + g + 8) * G::kGPitch + (8 * nt + 2 * c) * 2, ga[nt][1]);
       }
       if (a.dk) {
-        const int pos0 = sPos[st * kChunk + 16 * warp + g];
-        const int pos1 = sPos[st * kChunk + 16 * warp + g + 8];
-        float* dk0 = a.dk + ((int64_t)b * a.kv_len + (pos0 >= 0 ? pos0 : 0)) * DI;
-        float* dk1 = a.dk + ((int64_t)b * a.kv_len + (pos1 >= 0 ? pos1 : 0)) * DI;
+        // Even lanes of a pair add 4 columns of key g, odd lanes 4 columns of key g + 8.
+        const bool odd = c & 1;
+        const int pos = sPos[st * kChunk + 16 * warp + g + (odd ? 8 : 0)];
+        float* dkrow = a.dk + ((int64_t)b * a.kv_len + (pos >= 0 ? pos : 0)) * DI + 2 * (c & ~1);
 #pragma unroll
         for (int half = 0; half < (G::kNT + 7) / 8; ++half) {
           constexpr int kW = G::kNT < 8 ? G::kNT : 8;
@@ -351,9 +358,10 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_kl_kernel(const KLArgs a)
           }
 #pragma unroll
           for (int j = 0; j < kW; ++j) {
-            const int col = 8 * (half * 8 + j) + 2 * c;
-            if (pos0 >= 0) atomicAdd(reinterpret_cast<float2*>(dk0 + col), make_float2(acc[j][0], acc[j][1]));
-            if (pos1 >= 0) atomicAdd(reinterpret_cast<float2*>(dk1 + col), make_float2(acc[j][2], acc[j][3]));
+            const float r0 = __shfl_xor_sync(0xffffffffu, odd ? acc[j][0] : acc[j][2], 1);
+            const float r1 = __shfl_xor_sync(0xffffffffu, odd ? acc[j][1] : acc[j][3], 1);
+            const float4 v4 = odd ? make_float4(r0, r1, acc[j][2], acc[j][3]) : make_float4(acc[j][0], acc[j][1], r0, r1);
+            if (pos >= 0) atomicAdd(reinterpret_cast<float4*>(dkrow + 8 * (half * 8 + j)), v4);
           }
         }
       }
@@ -373,7 +381,6 @@ __global__ void __launch_bounds__(kThreads, 2) indexer_kl_kernel(const KLArgs a)
         }
       }
     }
-    __syncthreads();   // this stage and G are free again
   }
   cp_async_wait<0>();
   if (row_ok && !backward) row_ok = row_softmax_kl();

@@ -96,6 +96,21 @@ struct KLArgs {
   DeviceStatus* status;
 };
 
+// Sparse-stage teacher: head-summed, L1-normalised attention probabilities on
+// the selected set, from the forward's lse (attn_teacher.cu).
+constexpr int kMaxTeacherTopk = 4096;
+struct TeacherArgs {
+  int rows, nq, kv_len, H, Dqk, k;
+  float scale;
+  const uint16_t* q;           // [rows, H, Dqk] bf16
+  const uint16_t* latent;      // [B, kv_len, Dqk] bf16
+  const int32_t* idx;          // [rows, k]
+  const float* lse;            // [rows, H]
+  float* p_out;                // [rows, k]
+  DeviceStatus* status;
+  uint64_t timeout_ns;
+};
+
 cudaError_t launch_indexer_scan(int HI, bool fp8, int kblocks, const CUtensorMap& tq, const CUtensorMap& tk,
                                 const ScanArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_indexer_topk_prefill(int HI, bool fp8, int kblocks, const CUtensorMap& tq,
@@ -107,6 +122,8 @@ cudaError_t launch_fill_trivial_rows(int B, int nq, int q_offset, int rows_per_s
 cudaError_t launch_fill_f32(float* p, int64_t n, float v, cudaStream_t stream);
 cudaError_t launch_sparse_attn(const AttnArgs& a, int grid, cudaStream_t stream);
 size_t indexer_kl_smem_bytes(int dI, int k);
+size_t attn_teacher_smem_bytes(int k);
+cudaError_t launch_attn_teacher(const TeacherArgs& a, cudaStream_t stream);
 cudaError_t launch_indexer_kl(int dI, const KLArgs& a, cudaStream_t stream);
 cudaError_t launch_wait_selftest(DeviceStatus* status, uint64_t timeout_ns, cudaStream_t stream);
 cudaError_t launch_selection_overlap(int rows, int k, int max_pos, const int32_t* idx_a, const int32_t* idx_b,

@@ -7,10 +7,11 @@ is input preparation for the FP8 workload: each token's values are divided by
 a per-token scale (amax / 448) and rounded to FP8-e4m3 by torch's cast; the
 codes and the fp32 scales then *are* the inputs of both sides.
 
-Shapes and value distributions follow the five workloads the DSA path is
+Shapes and value distributions follow the workloads the DSA path is
 measured on (tiny integer prefill, integer prefill n=8192, FP8 prefill
-2x32768, decode batch 64 with ragged contexts 4096..65536, long prefill
-n=131072 in 8192-query chunks).  No dataset is involved.
+2x32768, decode batch 64 with ragged contexts 4096..65536 (bf16 or FP8 key
+cache), long prefill n=131072 in 8192-query chunks, and the sparse training
+stage's indexer KL on the n=8192 prefill).  No dataset is involved.
 """
 
 from __future__ import annotations
@@ -27,7 +28,7 @@ FP8_MAX = 448.0
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str                 # "prefill" or "decode"
+    kind: str                 # "prefill", "decode" or "train" (indexer KL, eq. (8))
     B: int
     n: int                    # tokens per sequence (prefill)
     HI: int                   # indexer heads
@@ -67,8 +68,12 @@ DECODE_FP8 = Workload("decode_fp8", "decode", B=64, n=0, HI=64, dI=128, k=2048, 
                       qk_dist="normal", w_std=0.1, fp8=True, seed=3, L_min=4096, L_max=65536)
 LONG = Workload("long_prefill", "prefill", B=1, n=131072, HI=64, dI=128, k=2048, H=16, Dqk=576,
                 Dv=512, qk_dist="normal", w_std=0.1, chunk=8192, seed=4)
+# Sparse training stage (eq. (8)): the prefill workload's inputs; the teacher
+# comes from the sparse attention on each row's selected set.
+INDEXER_KL = Workload("indexer_kl", "train", B=1, n=8192, HI=64, dI=128, k=2048, H=16, Dqk=576, Dv=512,
+                      qk_dist="int", qk_int_max=3, w_den=16, seed=1)
 
-ALL = {w.name: w for w in (TINY, PREFILL, PREFILL_FP8, DECODE, DECODE_FP8, LONG)}
+ALL = {w.name: w for w in (TINY, PREFILL, PREFILL_FP8, DECODE, DECODE_FP8, LONG, INDEXER_KL)}
 
 
 def scaled(w: Workload, **changes) -> Workload:

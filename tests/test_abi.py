@@ -134,3 +134,20 @@ def test_indexer_kl_argument_checks(lib):
     assert call(wsb=8) == 3
     assert call(nq=0) == 0                       # nothing to do
     assert lib.dsa_indexer_kl_workspace() == 256
+
+
+def test_attn_teacher_argument_checks(lib):
+    f = lib.dsa_attn_teacher_prefill
+    v = C.c_void_p(256)
+
+    def call(B=1, nq=4, kv_len=16, H=16, Dqk=576, k=8, scale=0.1, q=v, ws=v, wsb=256):
+        return f(B, nq, kv_len, H, Dqk, k, scale, q, v, v, v, v, ws, wsb, None)
+
+    assert call(Dqk=600) == 2                    # past the fixed 576-column row
+    assert call(Dqk=72) == 2                     # not a multiple of 16
+    assert call(k=4097) == 2
+    assert call(k=0) == 1
+    assert call(q=None) == 1
+    assert call(scale=float("nan")) == 1
+    assert call(wsb=8) == 3
+    assert call(nq=0) == 0
