@@ -9,12 +9,17 @@
 // order over CTAs.  Per CTA (18 warps):
 //   warp 0      TMA producer: Q of the block (both groups, once), K tiles;
 //   warp 1      tcgen05 MMA issuer, TMEM owner: for each 128-key tile and
-//               each group g of 4 tokens, D_g[128 keys x 4*HI] (+)= K Q_g^T;
-//   warps 2..17 epilogue, 4 warpgroups; warpgroup j takes token j of group 0
-//               and token 4+j of group 1 (both accumulators, in MMA order):
-//               TMEM -> ReLU * w -> head sum = I[t, s]; causal mask; then
-//               the streaming filter below; after the block's last tile the
-//               exact select (select.cuh) writes idx (and scores).
+//               each accumulator g, D_g[128 keys x T*HI] (+)= K Q_g^T, where
+//               an accumulator holds T = 2 tokens (four accumulators of 2*HI
+//               columns, one per epilogue warpgroup, when 2*HI >= 16) or
+//               T = 4 tokens (two accumulators shared by all warpgroups);
+//   warps 2..17 epilogue, 4 warpgroups; warpgroup j takes tokens 2j and
+//               2j+1 (four accumulators) or j and 4+j (two), in MMA order:
+//               TMEM -> ReLU * w -> head sum = I[t, s];
+//               causal mask; then the streaming filter below; an accumulator
+//               is released to the MMA issuer by the warpgroups that read it;
+//               after the block's last tile the exact select (select.cuh)
+//               writes idx (and scores).
 // Streaming filter, per token: a 512-bin histogram of accepted scores over a
 // monotone binning of the score (quarter-octaves for 2^-31 <= |x| < 2^31).
 // bin_floor only rises: once at least k accepted entries lie in bins above
