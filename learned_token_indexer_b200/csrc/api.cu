@@ -358,6 +358,7 @@ dsa_status dsa_indexer_topk_decode(int B, int HI, int dI, int k, int dtype, cons
   a.chunk_tiles = kScanChunkTiles;
   const int tiles = (max_len + 127) / 128;
   a.max_chunks = std::max(1, (tiles + kScanChunkTiles - 1) / kScanChunkTiles);
+  a.balanced = B <= dsa::kScanMaxBalancedRows ? 1 : 0;
   a.w = w;
   a.q_scale = fp8 ? q_scale : nullptr;
   a.k_scale = fp8 ? k_scale : nullptr;
@@ -417,6 +418,7 @@ dsa_status dsa_indexer_scores(int B, int nq, int q_offset, int kv_len, int HI, i
   a.chunk_tiles = kScanChunkTiles;
   const int tiles = (q_offset + nq + 127) / 128;
   a.max_chunks = std::max(1, (tiles + kScanChunkTiles - 1) / kScanChunkTiles);
+  a.balanced = 0;   // dense prefill rows: every row has max_chunks item slots
   a.w = w;
   a.q_scale = fp8 ? q_scale : nullptr;
   a.k_scale = fp8 ? k_scale : nullptr;

@@ -19,7 +19,11 @@ namespace dsa {
 
 namespace {
 
-constexpr int kScanStages = 4;
+// K tiles in flight: 128 KB of K^I per CTA whatever the tile size (a 128-byte
+// row tile, e4m3 or d^I = 64 bf16, needs twice as many tiles in flight as a
+// 256-byte one to keep the same bytes on the way from HBM).
+template <int KB>
+constexpr int scan_stages() { return KB == 1 ? 8 : 4; }
 constexpr int kScanThreads = 192;
 constexpr int kEpiWarp0 = 2;
 
@@ -46,15 +50,50 @@ __device__ __forceinline__ ScanRow scan_row(const ScanArgs& a, int r) {
 }
 
 // Item i -> (row, first tile, number of tiles); ntiles == 0 means empty.
+// Ragged decode rows (balanced mode) number only the non-empty chunks:
+// pre[r] = chunks of rows 0..r-1, so a persistent grid gets an even share of
+// the real work whatever the length mix; otherwise every row has max_chunks
+// item slots.
 __device__ __forceinline__ void scan_item(const ScanArgs& a, int item, int& row, int& t0, int& nt,
-                                          ScanRow& g) {
-  row = item / a.max_chunks;
-  const int c = item - row * a.max_chunks;
+                                          ScanRow& g, const int* pre, bool balanced) {
+  int c;
+  if (balanced) {
+    int lo = 0, hi = a.rows;   // pre[lo] <= item < pre[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pre[mid] <= item) lo = mid; else hi = mid;
+    }
+    row = lo;
+    c = item - pre[lo];
+  } else {
+    row = item / a.max_chunks;
+    c = item - row * a.max_chunks;
+  }
   g = scan_row(a, row);
   const int tiles = (g.len + kTileKeys - 1) / kTileKeys;
   t0 = c * a.chunk_tiles;
   nt = tiles - t0;
   nt = nt < 0 ? 0 : (nt > a.chunk_tiles ? a.chunk_tiles : nt);
+}
+
+// Eq. (1) for this thread's key: sum_j w_j * ReLU(D_j) with four independent
+// packed partial sums (the epilogue's critical path is this chain, one warp
+// per SM sub-partition), the weights read four at a time from shared memory.
+template <int HI>
+__device__ __forceinline__ float scan_head_sum(const uint32_t (&acc)[HI], const float* w_smem) {
+  static_assert(HI % 4 == 0, "heads come in fours");
+  float2 p[2][2] = {{make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)},
+                    {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)}};
+#pragma unroll
+  for (int j = 0; j < HI; j += 4) {
+    const float4 w4 = *reinterpret_cast<const float4*>(w_smem + j);
+    const float2 r0 = make_float2(fmaxf(__uint_as_float(acc[j]), 0.0f), fmaxf(__uint_as_float(acc[j + 1]), 0.0f));
+    const float2 r1 = make_float2(fmaxf(__uint_as_float(acc[j + 2]), 0.0f), fmaxf(__uint_as_float(acc[j + 3]), 0.0f));
+    const int c = (j >> 2) & 1;
+    p[c][0] = ffma2(make_float2(w4.x, w4.y), r0, p[c][0]);
+    p[c][1] = ffma2(make_float2(w4.z, w4.w), r1, p[c][1]);
+  }
+  return ((p[0][0].x + p[0][0].y) + (p[0][1].x + p[0][1].y)) + ((p[1][0].x + p[1][0].y) + (p[1][1].x + p[1][1].y));
 }
 
 }  // namespace
@@ -69,6 +108,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   constexpr uint32_t kTmemCols = (2 * N <= 32) ? 32 : (2 * N <= 64 ? 64 : (2 * N <= 128 ? 128 : 256));
   constexpr uint32_t kIdesc = instr_desc(ElemTraits<FP8>::kFormat, kTileKeys, N);
   constexpr int kElemsPerBlock = ElemTraits<FP8>::kElemsPerBlock;
+  constexpr int kScanStages = scan_stages<KB>();
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -85,6 +125,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   uint64_t* mma_done = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
+  int* sPre = reinterpret_cast<int*>(tmem_slot + 4);   // [rows + 1] in balanced mode
 
   const uint32_t warp = warp_id(), lane = lane_id();
   if (threadIdx.x == 0) {
@@ -110,12 +151,37 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  // balanced numbering needs the ragged offsets and room for the prefix
+  const bool balanced = a.balanced != 0 && a.mode == 1 && a.rows <= kScanMaxBalancedRows;
+  if (balanced) {
+    for (int r = threadIdx.x; r < a.rows; r += kScanThreads) {
+      const int64_t len = a.cu_seqlens[r + 1] - a.cu_seqlens[r];
+      const int tiles = (int)((len + kTileKeys - 1) / kTileKeys);
+      sPre[r + 1] = (tiles + a.chunk_tiles - 1) / a.chunk_tiles;
+    }
+    __syncthreads();
+    if (warp == 0) {   // inclusive scan of the chunk counts, 32 rows at a time
+      int carry = 0;
+      for (int r0 = 1; r0 <= a.rows; r0 += 32) {
+        const int r = r0 + (int)lane;
+        int v = r <= a.rows ? sPre[r] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= (uint32_t)o) v += u;
+        }
+        if (r <= a.rows) sPre[r] = carry + v;
+        carry += __shfl_sync(0xffffffffu, v, 31);
+      }
+      if (lane == 0) sPre[0] = 0;
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const WaitCtl ctl{abort_flag, a.timeout_ns, a.status};
-  const int total_items = a.rows * a.max_chunks;
+  const int total_items = balanced ? sPre[a.rows] : a.rows * a.max_chunks;
   const int ksteps = a.ksteps;
 
   if (warp == 0) {
@@ -131,7 +197,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
         int row, t0, nt;
         ScanRow g;
-        scan_item(a, item, row, t0, nt, g);
+        scan_item(a, item, row, t0, nt, g, sPre, balanced);
         if (nt == 0) continue;
         if (!(ok = mbar_wait(&q_empty[qslot], qphase ^ 1u, ctl, 0x101))) break;
         mbar_arrive_expect_tx(&q_full[qslot], kQBytes);
@@ -181,7 +247,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
         int row, t0, nt;
         ScanRow g;
-        scan_item(a, item, row, t0, nt, g);
+        scan_item(a, item, row, t0, nt, g, sPre, balanced);
         if (nt == 0) continue;
         if (!(ok = mbar_wait(&q_full[qslot], qphase, ctl, 0x201))) break;
         tc_fence_after();
@@ -219,7 +285,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
       int row, t0, nt;
       ScanRow g;
-      scan_item(a, item, row, t0, nt, g);
+      scan_item(a, item, row, t0, nt, g, sPre, balanced);
       if (nt == 0) continue;
       named_bar_sync(1, 128);
       if (et < (uint32_t)HI) {
@@ -229,6 +295,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       }
       named_bar_sync(1, 128);
       for (int t = 0; t < nt; ++t) {
+        const int s = (t0 + t) * kTileKeys + (int)lane_grp + (int)lane;
+        // the key's FP8 scale is requested before the wait, so its latency
+        // hides behind the MMA instead of following the head sum
+        float kscale = 1.0f;
+        if (FP8 && s < g.len) kscale = __ldg(a.k_scale + g.key_base + s);
         const bool got = ok && mbar_wait(&acc_full[acc], aphase, ctl, 0x301);
         ok = __all_sync(0xffffffffu, got);
         if (ok) {
@@ -239,10 +310,9 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[acc]);
-          const int s = (t0 + t) * kTileKeys + (int)lane_grp + (int)lane;
           if (s < g.len) {
-            float score = relu_weighted_head_sum<HI>(r, sW);
-            if (FP8) score *= a.k_scale[g.key_base + s];
+            float score = scan_head_sum<HI>(r, sW);
+            if (FP8) score *= kscale;
             g.out[s] = score + 0.0f;
           }
         }
@@ -261,8 +331,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 template <int HI, bool FP8, int KB>
 static size_t scan_smem_bytes() {
   constexpr int N = HI < 16 ? 16 : HI;
-  return 1024 + kScanStages * kTileKeys * KB * kSwizzleBytes + 2 * N * KB * kSwizzleBytes + 2 * HI * 4 +
-         (2 * kScanStages + 9) * 8 + 16;
+  return 1024 + scan_stages<KB>() * kTileKeys * KB * kSwizzleBytes + 2 * N * KB * kSwizzleBytes + 2 * HI * 4 +
+         (2 * scan_stages<KB>() + 9) * 8 + 16 + (kScanMaxBalancedRows + 1) * 4;
 }
 
 template <int HI, bool FP8, int KB>

@@ -9,6 +9,7 @@ namespace dsa {
 struct DeviceStatus;
 
 // Dense score rows (indexer_scan.cu).
+constexpr int kScanMaxBalancedRows = 4096;
 struct ScanArgs {
   int mode;                    // 0: prefill rows (b, i); 1: ragged decode rows
   int rows;                    // prefill B*nq; decode B
@@ -17,6 +18,7 @@ struct ScanArgs {
   int ksteps;                  // 32-byte MMA K steps holding data
   int chunk_tiles;             // key tiles per work item
   int max_chunks;              // work items per row (upper bound)
+  int balanced;                // decode: number only non-empty chunks (rows <= kScanMaxBalancedRows)
   const float* w;              // [rows, HI]
   const float* q_scale;        // [rows] (FP8) or null
   const float* k_scale;        // [key rows] (FP8) or null

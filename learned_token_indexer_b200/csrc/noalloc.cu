@@ -113,6 +113,7 @@ extern "C" dsa_status dsa_indexer_topk_decode_noalloc(int B, int HI, int dI, int
   a.chunk_tiles = kChunkTiles;
   const int tiles = (max_len + 127) / 128;
   a.max_chunks = (tiles + kChunkTiles - 1) / kChunkTiles > 0 ? (tiles + kChunkTiles - 1) / kChunkTiles : 1;
+  a.balanced = B <= dsa::kScanMaxBalancedRows ? 1 : 0;
   a.w = w;
   a.q_scale = fp8 ? q_scale : nullptr;
   a.k_scale = fp8 ? k_scale : nullptr;
