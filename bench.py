@@ -236,13 +236,46 @@ class PrefillRun:
         inter, cnt = dsa.selection_overlap(ref, self.idx, w.n, return_counts=True)
         torch.cuda.synchronize()
         ws.check()
-        rec = (inter.float() / cnt.clamp(min=1).float())[:, w.k:].flatten()
+        rec_all = inter.float() / cnt.clamp(min=1).float()
+        rec = rec_all[:, w.k:].flatten()
         q = torch.quantile(rec, torch.tensor([0.01, 0.5], device=rec.device))
-        return {"fp8_vs_bf16_recall": {"mean": round(float(rec.mean()), 5), "p01": round(float(q[0]), 5),
-                                       "median": round(float(q[1]), 5), "min": round(float(rec.min()), 5),
-                                       "rows": int(rec.numel()),
-                                       "definition": "|T ∩ S| / |T|, T = bf16 selection of the same draws, "
-                                                     "S = e4m3 selection; rows with t + 1 > k"}}
+        out = {"fp8_vs_bf16_recall": {"mean": round(float(rec.mean()), 5), "p01": round(float(q[0]), 5),
+                                      "median": round(float(q[1]), 5), "min": round(float(rec.min()), 5),
+                                      "rows": int(rec.numel()),
+                                      "definition": "|T ∩ S| / |T|, T = bf16 selection of the same draws, "
+                                                    "S = e4m3 selection; rows with t + 1 > k"}}
+        out["recall_by_margin"] = self._recall_by_margin(rec_all, ws)
+        return out
+
+    def _recall_by_margin(self, rec_all, ws, strip: int = 512, buckets: int = 4):
+        """Recall of the e4m3 selection grouped by the bf16 cut-off margin
+        Delta_k = s_(k) - s_(k+1) (eq. (18), §3.1: small margins are where a
+        perturbation swaps boundary tokens).  On the last `strip` rows of the
+        first sequence: dense bf16 scores (dsa_indexer_scores), their top
+        k + 1 (dsa_topk_rows), then quartiles of the margin."""
+        w, d, dsa = self.w, self.d, self.dsa
+        t0 = w.n - strip
+        sl = (slice(0, 1), slice(t0, w.n))
+        sc = dsa.indexer_scores(d["qI_bf16"][sl].contiguous(), d["kI_bf16"][:1].contiguous(),
+                                d["w"][sl].contiguous(), q_offset=t0, workspace=ws)[0]
+        row_len = torch.arange(t0 + 1, w.n + 1, dtype=torch.int32, device=sc.device)
+        _, val = dsa.topk_rows(sc, w.k + 1, row_len=row_len, return_values=True, workspace=ws)
+        torch.cuda.synchronize()
+        ws.check()
+        top = torch.sort(val, dim=1, descending=True).values
+        margin = (top[:, w.k - 1] - top[:, w.k]).double()
+        rec = rec_all[0, t0:].double()
+        edges = torch.quantile(margin, torch.linspace(0, 1, buckets + 1, dtype=torch.float64, device=margin.device))
+        rows = []
+        for i in range(buckets):
+            lo, hi = float(edges[i]), float(edges[i + 1])
+            m = (margin >= lo) & ((margin <= hi) if i == buckets - 1 else (margin < hi))
+            if int(m.sum()) == 0:
+                continue
+            rows.append({"margin": [round(lo, 6), round(hi, 6)], "rows": int(m.sum()),
+                         "mean_recall": round(float(rec[m].mean()), 5)})
+        return {"strip": f"rows {t0}..{w.n - 1} of sequence 0", "buckets": rows,
+                "definition": "Delta_k = s_(k) - s_(k+1) of the bf16 scores (eq. (18)); quartile buckets"}
 
     def kernel_work(self):
         w = self.w
