@@ -388,9 +388,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             if (lane == (uint32_t)(__ffs(peers) - 1)) atomicAdd(&sHist[st * kHistBins + bin], (uint32_t)__popc(peers));
           }
           cnt[u] += (uint32_t)__popc(mask);
-          // raise the floor (warp q = u of the group, every tile): the bin
-          // where the count of accepted scores from the top first reaches k
-          if (quarter == (uint32_t)u) raise_floor(sHist + st * kHistBins, (uint32_t)a.k, &sFloorKey[st], lane);
+          // raise the floor (every tile, by a warp that rotates with the
+          // tile so the four warps share the work): the bin where the count
+          // of accepted scores from the top first reaches k.  Two warps may
+          // raise one token's floor at once; each value written is a valid
+          // floor (counts only grow), so a lost update only admits more
+          if (quarter == ((uint32_t)(t + 2 * u) & 3u))
+            raise_floor(sHist + st * kHistBins, (uint32_t)a.k, &sFloorKey[st], lane);
         }
       }
       // per-warp candidate counts for the select
