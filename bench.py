@@ -291,7 +291,7 @@ class PrefillRun:
                                      "units": w.B * pairs},
             "sparse_attn": {"flops": 2 * w.H * w.B * ent * (w.Dqk + w.Dv), "unit": "TFLOP/s",
                             "per_unit": f"2*H*(Dqk+Dv) = {2 * w.H * (w.Dqk + w.Dv)} FLOP per selected entry",
-                            "units": w.B * ent},
+                            "units": w.B * ent, "gather_bytes": w.B * ent * w.Dqk * 2},
         }
 
     def host_inputs(self):
@@ -424,8 +424,9 @@ class TrainRun(PrefillRun):
                                      "units": w.B * pairs},
             "sparse_attn": {"flops": 2 * w.H * w.B * ent * (w.Dqk + w.Dv), "unit": "TFLOP/s",
                             "per_unit": f"2*H*(Dqk+Dv) = {2 * w.H * (w.Dqk + w.Dv)} FLOP per selected entry",
-                            "units": w.B * ent},
+                            "units": w.B * ent, "gather_bytes": w.B * ent * w.Dqk * 2},
             "attn_teacher": {"flops": 2 * w.H * w.B * ent * w.Dqk, "unit": "TFLOP/s",
+                             "gather_bytes": w.B * ent * w.Dqk * 2,
                              "per_unit": f"2*H*Dqk = {2 * w.H * w.Dqk} FLOP per selected entry (logits recompute)",
                              "units": w.B * ent},
             "indexer_kl": {"flops": 6 * w.HI * w.dI * w.B * ent, "unit": "TFLOP/s",
@@ -752,6 +753,11 @@ def run_b200(args):
                          "frac": round(ach / peak, 4), "ms_per_launch": round(t_launch, 4),
                          "traffic": measured_traffic(tkey, twl),
                          "algorithmic_per_launch": per_launch, "per_unit": wk["per_unit"]}
+        if "gather_bytes" in wk:
+            # the selected latent rows come from L2, not HBM: their rate is the
+            # secondary bound of the gathering kernels
+            kernels[name]["l2_gather_TBps"] = round(wk["gather_bytes"] / per_step_launches / (t_launch * 1e-3) / 1e12,
+                                                    3)
     dom = max(kernels, key=lambda n: kernels[n]["ms_per_launch"])
     roof = {k: kernels[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roof["kernel"] = dom
