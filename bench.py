@@ -7,7 +7,7 @@ the fused Lightning Indexer + causal top-k (eqs. (1)-(2) of the page
 "2.2.1 · DSA 与索引器") followed by sparse attention over the selected latent
 rows (eq. (3)).  The default workload is the integer-valued prefill
 (B=1, n=8192, HI=64, dI=128, k=2048, 16 heads, latent 576/512); the metric is
-query tokens per second.  --workload decode|prefill_fp8|long_prefill|tiny
+query tokens per second.  --workload decode|decode_fp8|prefill_fp8|long_prefill|tiny
 selects the other workloads; --workload indexer_kl times the sparse training
 stage's indexer step instead: selection, the sparse attention forward with
 its lse, the teacher recomputed on the selected set, then the eq. (8) KL on
@@ -18,6 +18,11 @@ on the launching stream; L2 is flushed (a 256 MiB write) before every timed
 step, outside the events.  Per-kernel events give the roofline of the
 dominant kernel.  Under torchrun every rank runs its own batch (weak
 scaling, no collective on the data path); rank 0 prints the max over ranks.
+
+End to end (`e2e`): every step uploads its inputs from pinned host memory,
+runs through the public API and downloads its result; timed both one step
+after another on one stream and with consecutive steps overlapped on three
+streams (two replicas of the device buffers), reporting the faster.
 
 --impl reference times the CPU oracle (float64 numpy) on a bounded sample of
 the same workload on the host cores.
