@@ -158,9 +158,10 @@ dsa_status dsa_indexer_topk_decode(int B, int HI, int dI, int k, int dtype, cons
  *   the library holds until the process exits.  Nothing is allocated.
  *   Limit: total_len <= 4,194,304 (2^22) cached keys over all B sequences;
  *   larger steps return DSA_ERR_UNSUPPORTED with a message naming the limit.
- *   Set-up: the first call made with a given device current looks up that
- *   device's copy of the buffer (a host-side step); make that first call
- *   before any stream capture.
+ *   Set-up: every call looks up the current device's copy of the buffer
+ *   with cudaGetSymbolAddress (a host-side step, so a device reset between
+ *   calls is harmless); the first call on a device also loads the library's
+ *   module there, so make that first call before any stream capture.
  *   Sharing: every call uses the same buffer, which keeps the last call's
  *   contents; the status word is cleared at the start of each call (the
  *   scores are fully rewritten).  Calls whose work overlaps on the GPU (two

@@ -10,7 +10,6 @@
 // into the library: a file-scope __device__ array, which every GPU that loads
 // the library holds until the process exits.  Nothing here allocates.
 #include <cstdio>
-#include <mutex>
 
 #include "dsa.h"
 #include "kernels.h"
@@ -21,15 +20,11 @@ namespace {
 constexpr int64_t kMaxKeys = int64_t(1) << 22;   // cached keys per call, all sequences together
 constexpr size_t kHeaderBytes = 256;             // device status word, then the scores
 constexpr size_t kScratchBytes = kHeaderBytes + size_t(kMaxKeys) * sizeof(float);   // 16 MiB + 256 B
-constexpr int kMaxDevices = 64;
 constexpr int kChunkTiles = 8;
 
 // In host code this name is only a stand-in for the device array: its device
-// address comes from cudaGetSymbolAddress, once per device (below).
+// address comes from cudaGetSymbolAddress, looked up on every call (below).
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
-
-std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
 
 dsa_status fail(dsa_status st, const char* msg) {
   dsa::set_last_error(msg);
@@ -42,25 +37,21 @@ dsa_status launch_fail(cudaError_t e, const char* what) {
   return fail(DSA_ERR_CUDA, msg);
 }
 
-// Device address of the built-in scratch on the current device (set up on the
-// first call made with that device current).
+// Device address of the built-in scratch on the current device.  It is looked
+// up on every call rather than cached: after a context teardown
+// (cudaDeviceReset) the module is loaded again and the array may sit at
+// another address, so a cached pointer would go stale.  The lookup is a host
+// call; the first one on a device also loads this library's module there.
 dsa_status scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-    return fail(DSA_ERR_CUDA, "dsa_indexer_topk_decode_noalloc: no usable current device");
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess || p == nullptr) {
-      char msg[256];
-      snprintf(msg, sizeof(msg), "dsa_indexer_topk_decode_noalloc: cudaGetSymbolAddress failed: %s",
-               cudaGetErrorString(e));
-      return fail(DSA_ERR_CUDA, msg);
-    }
-    g_scratch_addr[dev] = p;
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  if (e != cudaSuccess || p == nullptr) {
+    char msg[256];
+    snprintf(msg, sizeof(msg), "dsa_indexer_topk_decode_noalloc: cudaGetSymbolAddress failed: %s",
+             cudaGetErrorString(e));
+    return fail(DSA_ERR_CUDA, msg);
   }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return DSA_OK;
 }
 

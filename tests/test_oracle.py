@@ -51,6 +51,40 @@ def test_e4m3_decode_matches_torch_cast():
     assert np.array_equal(got[finite], ref[finite])
 
 
+def test_dequantize_scales_each_token_group():
+    """Dequantised value = code value x the scale of its token (§2: quantised
+    indexer key cache with its scales).  Keys carry one scale per key over
+    d^I (one trailing axis); queries one scale per token over H^I x d^I (two
+    trailing axes).  Scales are distinct and neither 1 nor self-reciprocal,
+    so a scale divided instead of multiplied, or broadcast over the head axis
+    instead of the token axis, changes the values checked here."""
+    # codes 0x38 = 1.0, 0x40 = 2.0, 0xB0 = -0.5, 0x00 = 0.0, 0x44 = 3.0
+    one, two, mhalf, zero, three = 0x38, 0x40, 0xB0, 0x00, 0x44
+    keys = np.array([[one, two, mhalf], [three, zero, one]], dtype=np.uint8)      # [2 keys, 3 dims]
+    kscale = np.array([0.25, 3.0])
+    got = O.dequantize(keys, kscale, 1)
+    assert got.shape == (2, 3)
+    assert got.tolist() == [[0.25, 0.5, -0.125], [9.0, 0.0, 3.0]]
+
+    # queries [3 tokens, 2 heads, 2 dims]; the head count (2) differs from the
+    # token count (3), and token 1's scale differs from head 1's position
+    q = np.array([[[one, two], [three, mhalf]],
+                  [[one, one], [two, zero]],
+                  [[mhalf, three], [one, two]]], dtype=np.uint8)
+    qscale = np.array([2.0, 0.125, 5.0])
+    got = O.dequantize(q, qscale, 2)
+    assert got.shape == (3, 2, 2)
+    want = [[[2.0, 4.0], [6.0, -1.0]],
+            [[0.125, 0.125], [0.25, 0.0]],
+            [[-2.5, 15.0], [5.0, 10.0]]]
+    assert got.tolist() == want
+    # leading batch axis: [B=2, tokens=3] scales over [B, tokens, H, d] codes
+    got_b = O.dequantize(np.stack([q, q]), np.stack([qscale, qscale[::-1]]), 2)
+    assert got_b[0].tolist() == want
+    assert got_b[1, 0].tolist() == (np.array(want[0]) / 2.0 * 5.0).tolist()
+    assert got_b[1, 2].tolist() == (np.array(want[2]) / 5.0 * 2.0).tolist()
+
+
 # --------------------------------------------------------------------------
 # Worked example of §1.1 (eqs. (4)-(6) and the text after them)
 # --------------------------------------------------------------------------
