@@ -320,6 +320,14 @@ dsa_status dsa_sparse_attn_decode(int B, int H, int Dqk, int Dv, int k, float sc
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
   a.status = status_of(workspace);
+  if (H == 128 && Dqk == 576 && Dv == 512 && aligned(out, 16)) {
+    // the MQA shape of the decode step: all 128 heads on the tensor-core M
+    DSA_CHECK(total_len < INT32_MAX && (int64_t)B * 2 <= INT32_MAX, DSA_ERR_UNSUPPORTED, "tensor rows exceed 2^31");
+    a.timeout_ns = g_timeout_ns;
+    cudaError_t e = dsa::launch_latent_attn_decode(a, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "latent_attn_decode launch");
+    return DSA_OK;
+  }
   return run_attn(a, q, latent_cache, total_len, (cudaStream_t)stream);
 }
 

@@ -123,6 +123,10 @@ cudaError_t launch_fill_trivial_rows(int B, int nq, int q_offset, int rows_per_s
                                      cudaStream_t stream);
 cudaError_t launch_fill_f32(float* p, int64_t n, float v, cudaStream_t stream);
 cudaError_t launch_sparse_attn(const AttnArgs& a, int grid, cudaStream_t stream);
+// Decode attention with 128 heads on the tcgen05 M (latent_attn_decode.cu):
+// H = 128, Dqk = 576, Dv = 512; one 2-CTA cluster per sequence (a.rows).
+cudaError_t launch_latent_attn_decode(const AttnArgs& a, cudaStream_t stream);
+size_t latent_attn_decode_smem();
 size_t indexer_kl_smem_bytes(int dI, int k);
 size_t attn_teacher_smem_bytes(int k);
 cudaError_t launch_attn_teacher(const TeacherArgs& a, cudaStream_t stream);

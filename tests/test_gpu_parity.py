@@ -362,6 +362,52 @@ def test_decode_fp8_cache_small_ragged():
     _decode_case(w, torch.tensor([1, 129, 300, 1000, 4097]))
 
 
+def test_decode_attention_scattered_and_bad_slots():
+    """The decode step's attention (128 heads, 576/512 latent rows: the
+    tensor-core kernel whose two CTAs split the latent columns) on ragged
+    sequences whose index rows hold -1 anywhere, a row with one usable slot,
+    an empty row and an index past the sequence end, which is reported and
+    skipped."""
+    g = torch.Generator().manual_seed(12)
+    lengths = torch.tensor([3000, 1, 700, 2500, 64, 129])
+    B, H, k, Dqk, Dv = lengths.numel(), 128, 640, 576, 512
+    cu = torch.zeros(B + 1, dtype=torch.int64)
+    cu[1:] = torch.cumsum(lengths, 0)
+    total = int(cu[-1])
+    q = torch.randn((B, H, Dqk), generator=g).bfloat16().cuda()
+    lat = torch.randn((total, Dqk), generator=g).bfloat16().cuda()
+    idx = torch.full((B, k), -1, dtype=torch.int32)
+    for b in range(B):
+        L = int(lengths[b])
+        m = min(k, L)
+        idx[b, :m] = torch.randperm(L, generator=g)[:m].int()
+        drop = torch.rand(k, generator=g) < 0.3
+        idx[b, drop] = -1                       # unused slots anywhere in the row
+    idx[1] = -1
+    idx[1, 5] = 0                               # one usable slot, not the first
+    idx[4] = -1                                 # nothing selected
+    bad = idx.clone()
+    bad[2, 77] = int(lengths[2]) + 3            # past the end of sequence 2
+    ws = _ws()
+    out, lse = dsa.sparse_attn_decode(q, lat, cu.cuda(), bad.cuda(), Dv, total, scale=1 / 24, return_lse=True,
+                                      workspace=ws)
+    st, detail = ws.status()
+    assert st == 6 and detail == 0xA77E
+    fixed = bad.clone()
+    fixed[2, 77] = -1
+    ro, rl = O.decode_sparse_attention(host_f64(q), host_f64(lat), cu.numpy(), fixed.numpy(), 1 / 24, Dv)
+    o, l_ = host_f64(out), lse.cpu().double().numpy()
+    assert np.all(o[4] == 0) and np.all(np.isneginf(l_[4]))
+    errs = checks.close_errors(o, ro, ATOL, RTOL, "decode out") + checks.close_errors(l_, rl, 1e-3, 1e-3, "lse")
+    assert not errs, errs
+    # the same call twice gives the same bits (no state kept between launches)
+    out2 = dsa.sparse_attn_decode(q, lat, cu.cuda(), fixed.cuda(), Dv, total, scale=1 / 24, workspace=ws)
+    out3 = dsa.sparse_attn_decode(q, lat, cu.cuda(), fixed.cuda(), Dv, total, scale=1 / 24, workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    assert torch.equal(out2, out3)
+
+
 @pytest.mark.slow
 def test_decode_full_workload():
     _decode_case(W.DECODE, W.decode_lengths(W.DECODE))
