@@ -8,7 +8,7 @@ helper with the CUDA library.
 Source: the page "2.2.1 · DSA 与索引器: 先召回 token, 再计算 Sparse MLA"
 (called "the DSA page" below), §1.1 eqs. (1)-(6), §1.2 eqs. (8) and (16)
 (sparse-stage indexer KL and its teacher), §2 (decode, quantised indexer key
-cache) and §3.1 eqs. (14), (18), §3.2 eqs. (19)-(20).
+cache) and §3.1 eqs. (14), (15), (18), §3.2 eqs. (19)-(20).
 
 Everything is float64 numpy.  Inputs are converted exactly to float64 first:
 bf16 values are exact in float64, and FP8-e4m3 codes are decoded by
@@ -55,6 +55,8 @@ __all__ = [
     "indexer_topk",
     "selection_stats_row",
     "selection_recall_row",
+    "mass_coverage_row",
+    "mass_coverage",
     "sparse_attention_row",
     "sparse_attention",
     "decode_indexer_topk",
@@ -204,6 +206,52 @@ def selection_recall_row(teacher_row, student_row) -> float:
     if not t:
         return 1.0
     return len(t & s) / len(t)
+
+
+def mass_coverage_row(q_t, latent_hist, sel, scale: float) -> dict:
+    """Teacher probability mass covered by a selection, eq. (15) of the DSA
+    page §3.1:  M_k = sum_{j in S_k} a_{tj}.
+
+    a_{tj} is the dense attention probability of the main attention over the
+    whole causal history 0..t (the teacher); with several query heads each
+    head h has its own a^(h) and the teacher the DSA report uses is their sum
+    over heads, L1-normalised along the sequence (eq. (16) with equal
+    weights), i.e. the mean over heads.  The page also asks for the lowest
+    per-head coverage, so both are returned.
+
+    q_t: [H, Dqk] query heads of token t; latent_hist: [t+1, Dqk] latent rows
+    0..t (the key is the whole row, as in eq. (3)); sel: selected positions,
+    -1 entries ignored.  Returns {"M": float, "per_head": [H], "min": float}.
+    """
+    q_t = _f64(q_t)
+    latent_hist = _f64(latent_hist)
+    sel = np.asarray(sel, dtype=np.int64)
+    sel = np.unique(sel[sel >= 0])
+    z = scale * (q_t @ latent_hist.T)               # [H, t+1] dense logits
+    e = np.exp(z - z.max(axis=1, keepdims=True))
+    a = e / e.sum(axis=1, keepdims=True)            # a^(h)_{tj}, each row sums to 1
+    per_head = a[:, sel].sum(axis=1)                # coverage of each head
+    p = a.sum(axis=0)                               # sum over heads ...
+    p = p / p.sum()                                 # ... L1-normalised along the sequence
+    return {"M": float(p[sel].sum()), "per_head": per_head, "min": float(per_head.min())}
+
+
+def mass_coverage(q, latent, idx, scale: float, q_offset: int = 0, rows=None) -> dict:
+    """``mass_coverage_row`` for a prefill chunk: q [B, nq, H, Dqk], latent
+    [B, kv_len, Dqk], idx [B, nq, k]; row i sits at t = q_offset + i.
+    Returns M [B, nq], per_head [B, nq, H] and min [B, nq] (NaN in rows left
+    out by ``rows``)."""
+    q = _f64(q)
+    latent = _f64(latent)
+    idx = np.asarray(idx.cpu() if hasattr(idx, "cpu") else idx, dtype=np.int64)
+    B, nq, H = q.shape[0], q.shape[1], q.shape[2]
+    out = {"M": np.full((B, nq), np.nan), "per_head": np.full((B, nq, H), np.nan), "min": np.full((B, nq), np.nan)}
+    todo = rows if rows is not None else [(b, i) for b in range(B) for i in range(nq)]
+    for b, i in todo:
+        t = q_offset + i
+        r = mass_coverage_row(q[b, i], latent[b, : t + 1], idx[b, i], scale)
+        out["M"][b, i], out["per_head"][b, i], out["min"][b, i] = r["M"], r["per_head"], r["min"]
+    return out
 
 
 def indexer_topk(q, k, w, topk: int, q_offset: int = 0, rows=None) -> np.ndarray:

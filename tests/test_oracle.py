@@ -343,6 +343,110 @@ def test_sparse_renormalisation_identity_and_bound():
     assert np.linalg.norm(dense[0] - sparse[0]) <= 2 * (1 - M) * V + 1e-12
 
 
+# --------------------------------------------------------------------------
+# Eq. (15): teacher probability mass covered by a selection
+# --------------------------------------------------------------------------
+
+def _single_head_latents(logits):
+    """Latent rows whose logits against q = e_0 (scale 1) are `logits`."""
+    lat = np.zeros((len(logits), 4))
+    lat[:, 0] = logits
+    lat[:, 1:] = np.arange(1, len(logits) + 1)[:, None] * np.array([0.5, -1.0, 2.0])
+    return np.array([[1.0, 0.0, 0.0, 0.0]]), lat
+
+
+def test_mass_coverage_worked_example_miss_case():
+    """§1.1 miss case: full logits 0.2, 1.2, 2.0 at positions 1, 2, 3 and the
+    selector returned {1, 2}: the covered mass is the closed form
+    (e^0.2 + e^1.2) / (e^0.2 + e^1.2 + e^2.0); selecting all three covers 1."""
+    g = _worked()
+    logits = g["attention_logits"] + [g["miss_case_logit_position3"]]
+    q, lat = _single_head_latents(logits)
+    r = O.mass_coverage_row(q, lat, np.array(g["selected_positions_0based"]), 1.0)
+    want = (math.exp(0.2) + math.exp(1.2)) / (math.exp(0.2) + math.exp(1.2) + math.exp(2.0))
+    assert abs(r["M"] - want) < 1e-15 and abs(r["per_head"][0] - want) < 1e-15
+    assert abs(r["M"] - 0.3807) < 1e-4           # the missed top position held ~62% of the mass
+    full = O.mass_coverage_row(q, lat, np.array([2, 0, 1, -1]), 1.0)
+    assert abs(full["M"] - 1.0) < 1e-15
+
+
+def test_mass_coverage_renormalisation_factor_from_the_page():
+    """§3.2 after eq. (19): with M_k = 0.6 the retained positions are scaled by
+    1/M_k ~ 1.67, with M_k = 0.98 by ~1.02.  Build dense probabilities with
+    exactly that retained mass and check both M_k and eq. (19)'s rescaling of
+    the sparse output."""
+    for kept, factor in ((0.6, 1.67), (0.98, 1.02)):
+        a = np.array([kept / 2, kept / 2, (1 - kept) / 3, (1 - kept) / 3, (1 - kept) / 3])
+        q, lat = _single_head_latents(np.log(a))
+        r = O.mass_coverage_row(q, lat, np.array([0, 1]), 1.0)
+        assert abs(r["M"] - kept) < 1e-12
+        assert abs(1.0 / r["M"] - factor) < 5e-3
+        sparse, _ = O.sparse_attention_row(q, lat, np.array([0, 1]), 1.0, 4)
+        renorm = (a[:2, None] / r["M"] * lat[:2, :4]).sum(axis=0)
+        assert np.allclose(sparse[0], renorm, atol=1e-12)
+
+
+def test_mass_coverage_per_head_and_eq19_identity():
+    """Per head, the sparse output equals sum_{j in S} a_j^(h) v_j / m_h with m_h
+    the head's covered mass (eq. (19)); the aggregate M is the mean over heads
+    of m_h (sum over heads, then L1 along the sequence, eq. (16))."""
+    rng = np.random.default_rng(15)
+    H, t1, Dqk, Dv = 3, 23, 10, 6
+    q = rng.standard_normal((H, Dqk))
+    lat = rng.standard_normal((t1, Dqk)) * 1.3
+    sel = rng.choice(t1, 9, replace=False)
+    r = O.mass_coverage_row(q, lat, sel, 0.7)
+    sparse, _ = O.sparse_attention_row(q, lat, sel, 0.7, Dv)
+    for h in range(H):
+        z = 0.7 * (lat @ q[h])
+        a = np.exp(z - z.max())
+        a /= a.sum()
+        assert abs(r["per_head"][h] - a[sel].sum()) < 1e-13
+        assert np.allclose(sparse[h], (a[sel, None] * lat[sel, :Dv]).sum(axis=0) / r["per_head"][h], atol=1e-12)
+    assert abs(r["M"] - r["per_head"].mean()) < 1e-13
+    assert abs(r["min"] - r["per_head"].min()) < 1e-15
+    # slot order, -1 padding and a repeated position do not change the set
+    r2 = O.mass_coverage_row(q, lat, np.concatenate([sel[::-1], [-1, sel[0]]]), 0.7)
+    assert abs(r2["M"] - r["M"]) < 1e-14
+
+
+def test_mass_coverage_three_heads_cannot_share_two_slots():
+    """§3.1 three-head example: heads put 0.9 of their mass on positions 10,
+    20 and 30, budget k = 2.  Every shared pair leaves one head with at most
+    the remaining 0.1 of its mass, while the mean coverage stays ~0.63."""
+    n = 40
+    peaks = (10, 20, 30)
+    a = np.full((3, n), 0.1 / (n - 1))
+    for h, pos in enumerate(peaks):
+        a[h, pos] = 0.9
+    # logits realising these probabilities (q_h = e_h, latent column h = log a_h)
+    lat = np.zeros((n, 3))
+    lat[:, :] = np.log(a).T
+    q = np.eye(3)
+    for pair in ((10, 20), (10, 30), (20, 30)):
+        r = O.mass_coverage_row(q, lat, np.array(pair), 1.0)
+        assert r["min"] < 0.1 + 1e-12
+        assert abs(r["M"] - (2 * 0.9 + 3 * 0.1 / (n - 1) * 2 - 0.1 / (n - 1) * 2) / 3) < 1e-12
+        assert np.sum(r["per_head"] > 0.9 - 1e-12) == 2
+
+
+def test_mass_coverage_brute_force_small():
+    """Explicit loops with Python floats on a tiny two-head case."""
+    rng = np.random.default_rng(16)
+    H, t1, Dqk = 2, 6, 3
+    q = rng.integers(-2, 3, (H, Dqk)).astype(float)
+    lat = rng.integers(-2, 3, (t1, Dqk)).astype(float)
+    sel = [4, 1, 5]
+    scale = 0.5
+    per = []
+    for h in range(H):
+        ez = [math.exp(scale * sum(q[h, d] * lat[j, d] for d in range(Dqk))) for j in range(t1)]
+        per.append(sum(ez[j] for j in sel) / sum(ez))
+    r = O.mass_coverage_row(q, lat, np.array(sel), scale)
+    assert np.allclose(r["per_head"], per, atol=1e-14)
+    assert abs(r["M"] - sum(per) / H) < 1e-14
+
+
 def test_attention_ignores_padding_and_slot_order():
     rng = np.random.default_rng(9)
     lat = rng.standard_normal((30, 8))
