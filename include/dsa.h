@@ -128,6 +128,43 @@ dsa_status dsa_sparse_attn_prefill(int B, int nq, int kv_len, int H, int Dqk, in
                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Dense masked attention, prefill  (§2, the short-prefill paragraph: for
+ * short sequences the fixed costs of top-k, index materialisation and the
+ * irregular gather exceed the attention they save, and DSA is run as masked
+ * MHA instead; the serving side picks the path by length).  Same result as
+ * dsa_sparse_attn_prefill on the same selection (eq. (3), §1.1), computed
+ * over dense causal key tiles that a block of 8 tokens shares:
+ *   row i of sequence b (absolute position t = q_offset + i) attends the
+ *   keys s <= t; if idx is given and t + 1 > k it attends only the
+ *   positions its row of idx selects (rows with t + 1 <= k select every
+ *   position, eq. (2)); with idx NULL it is plain causal attention over the
+ *   whole history, whose lse is the dense normaliser of eq. (15).
+ *   q [B, nq, 16, 576] bf16   latent [B, kv_len, 576] bf16 (rows 0..kv_len-1)
+ *   idx [B, nq, k] int32 (positions in [0, kv_len) or -1) or NULL
+ *   out [B, nq, 16, 512] bf16   lse [B, nq, 16] fp32 or NULL
+ * Workspace: dsa_attn_dense_prefill_workspace(B, nq, kv_len, idx != NULL)
+ * bytes (the status header, plus one selection bit per (row, key) when idx
+ * is given).  An index outside [-1, kv_len) is skipped and recorded as
+ * DSA_ERR_DEVICE_CHECK (0xA77E).  Supported: H = 16, Dqk = 576, Dv = 512;
+ * q, latent and out 16-byte aligned; q_offset + nq <= kv_len.
+ * ---------------------------------------------------------------------- */
+size_t dsa_attn_dense_prefill_workspace(int B, int nq, int kv_len, int with_selection);
+dsa_status dsa_attn_dense_prefill(int B, int nq, int q_offset, int kv_len, int H, int Dqk, int Dv, int k, float scale,
+                                  const void* q, const void* latent, const int32_t* idx, void* out, float* lse,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Teacher mass coverage of a selection (§3.1, eq. (15)): for each of `rows`
+ * query rows and each head h, the dense attention probabilities on the
+ * selected positions sum to exp(lse_sparse[r, h] - lse_dense[r, h]) (the lse
+ * outputs of the sparse attention over the selection and of the dense causal
+ * attention); the teacher of eq. (16) (heads summed, L1-normalised) covers
+ * their mean.  lse_sparse, lse_dense [rows, H] fp32 device arrays; outputs
+ * (each may be NULL): m_out [rows] the aggregate M_k, per_head_out [rows, H],
+ * min_out [rows] the lowest per-head coverage.  Needs no workspace. */
+dsa_status dsa_mass_coverage(int rows, int H, const float* lse_sparse, const float* lse_dense, float* m_out,
+                             float* per_head_out, float* min_out, void* stream);
+
+/* ------------------------------------------------------------------------
  * Decode step  (§2: one new query per sequence scans every cached indexer
  * key; the latent cache is shared by all query heads, MQA form).
  * Ragged caches: sequence b owns rows cu_seqlens[b] .. cu_seqlens[b+1]-1 of

@@ -167,6 +167,47 @@ def sparse_attn_prefill(q, latent, idx, dv: int, scale: Optional[float] = None, 
     return (out, lse) if lse is not None else out
 
 
+def attn_dense_prefill(q, latent, dv: int, idx=None, k: Optional[int] = None, q_offset: int = 0,
+                       scale: Optional[float] = None, out=None, lse=None, return_lse: bool = False,
+                       workspace: Optional[Workspace] = None):
+    """Eq. (3) over dense causal key tiles (§2, short prefill as masked MHA):
+    q [B, nq, 16, 576], latent [B, kv_len, 576]; with idx [B, nq, k] the rows
+    with t + 1 > k see only their selection (the same result as
+    sparse_attn_prefill), without it every causal key (the dense attention
+    whose lse normalises eq. (15))."""
+    B, nq, H, Dqk = q.shape
+    kv_len = latent.shape[1]
+    if idx is not None:
+        k = idx.shape[-1] if k is None else k
+    scale = Dqk ** -0.5 if scale is None else scale
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, nq, H, dv), dtype=torch.bfloat16, device=dev)
+    if return_lse and lse is None:
+        lse = torch.empty((B, nq, H), dtype=torch.float32, device=dev)
+    L = lib()
+    wsb = _ws(workspace, dev).get(L.dsa_attn_dense_prefill_workspace(B, nq, kv_len, 1 if idx is not None else 0))
+    _check(L.dsa_attn_dense_prefill(B, nq, q_offset, kv_len, H, Dqk, dv, int(k or 0), float(scale), _ptr(q),
+                                    _ptr(latent), _ptr(idx), _ptr(out), _ptr(lse), _ptr(wsb), wsb.numel(),
+                                    _stream(dev)))
+    return (out, lse) if lse is not None else out
+
+
+def mass_coverage(lse_sparse, lse_dense, per_head: bool = False):
+    """Teacher mass coverage M_k of eq. (15) per query row from the two lse
+    tensors [..., H]: returns (M, min over heads) [...] (and the per-head
+    coverage [..., H] with per_head=True)."""
+    H = lse_sparse.shape[-1]
+    rows = lse_sparse.numel() // H
+    dev = lse_sparse.device
+    m = torch.empty(lse_sparse.shape[:-1], dtype=torch.float32, device=dev)
+    mn = torch.empty_like(m)
+    ph = torch.empty_like(lse_sparse) if per_head else None
+    _check(lib().dsa_mass_coverage(rows, H, _ptr(lse_sparse), _ptr(lse_dense), _ptr(m), _ptr(ph), _ptr(mn),
+                                   _stream(dev)))
+    return (m, mn, ph) if per_head else (m, mn)
+
+
 # --------------------------------------------------------------------------
 # Decode
 # --------------------------------------------------------------------------

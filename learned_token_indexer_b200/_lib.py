@@ -32,6 +32,9 @@ SIGNATURES = {
     "dsa_selftest_bounded_wait": (_i, [_u64, _p, _sz, _p]),
     "dsa_selection_overlap": (_i, [_i, _i, _i, _p, _p, _p, _p, _p]),
     "dsa_indexer_kl_workspace": (_sz, []),
+    "dsa_attn_dense_prefill_workspace": (_sz, [_i, _i, _i, _i]),
+    "dsa_attn_dense_prefill": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "dsa_mass_coverage": (_i, [_i, _i, _p, _p, _p, _p, _p, _p]),
     "dsa_attn_teacher_prefill": (_i, [_i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "dsa_indexer_kl_sparse": (_i, [_i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _f, _p, _p, _p, _p, _p, _p, _sz, _p]),
 }

@@ -331,6 +331,62 @@ dsa_status dsa_sparse_attn_decode(int B, int H, int Dqk, int Dv, int k, float sc
   return run_attn(a, q, latent_cache, total_len, (cudaStream_t)stream);
 }
 
+// ---------------------------------------------------------------- dense masked attention
+size_t dsa_attn_dense_prefill_workspace(int B, int nq, int kv_len, int with_selection) {
+  if (!with_selection || B <= 0 || nq <= 0 || kv_len <= 0) return kHeader;
+  return kHeader + round_up((size_t)B * nq * (size_t)((kv_len + 63) / 64) * sizeof(uint64_t), 256);
+}
+
+dsa_status dsa_attn_dense_prefill(int B, int nq, int q_offset, int kv_len, int H, int Dqk, int Dv, int k, float scale,
+                                  const void* q, const void* latent, const int32_t* idx, void* out, float* lse,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  DSA_CHECK(H == 16 && Dqk == 576 && Dv == 512, DSA_ERR_UNSUPPORTED,
+            "dense attention supports H=16, Dqk=576, Dv=512 (got H=%d Dqk=%d Dv=%d)", H, Dqk, Dv);
+  DSA_CHECK(B >= 1 && nq >= 0 && q_offset >= 0 && kv_len >= 1 && (int64_t)q_offset + nq <= kv_len,
+            DSA_ERR_INVALID_ARG, "need B >= 1, nq >= 0, q_offset >= 0, q_offset + nq <= kv_len");
+  DSA_CHECK(idx == nullptr || k >= 1, DSA_ERR_INVALID_ARG, "k must be >= 1 with an index tensor");
+  DSA_CHECK(std::isfinite(scale), DSA_ERR_INVALID_ARG, "scale must be finite");
+  DSA_CHECK((int64_t)B * kv_len < INT32_MAX && (int64_t)B * nq * H < INT32_MAX, DSA_ERR_UNSUPPORTED,
+            "tensor rows exceed 2^31");
+  DSA_CHECK(q && latent && out, DSA_ERR_INVALID_ARG, "null tensor pointer");
+  DSA_CHECK(aligned(q, 16) && aligned(latent, 16) && aligned(out, 16) && aligned(idx, 4) && aligned(lse, 4),
+            DSA_ERR_INVALID_ARG, "q, latent and out must be 16-byte aligned");
+  const size_t need = dsa_attn_dense_prefill_workspace(B, nq, kv_len, idx != nullptr);
+  if (dsa_status st = check_ws(workspace, workspace_bytes, need)) return st;
+  if (nq == 0) return DSA_OK;
+  dsa::DenseAttnArgs a{};
+  a.B = B;
+  a.nq = nq;
+  a.q_offset = q_offset;
+  a.kv_len = kv_len;
+  a.k = idx ? k : 0;
+  a.nblk = (nq + 7) / 8;
+  a.kv_tiles = (kv_len + 63) / 64;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.q = static_cast<const uint16_t*>(q);
+  a.sel_bits = idx ? reinterpret_cast<const uint64_t*>(static_cast<char*>(workspace) + kHeader) : nullptr;
+  a.out = static_cast<uint16_t*>(out);
+  a.lse = lse;
+  a.status = status_of(workspace);
+  a.timeout_ns = g_timeout_ns;
+  DSA_CHECK((int64_t)B * a.nblk * 2 < INT32_MAX, DSA_ERR_UNSUPPORTED, "too many token blocks");
+  CUtensorMap tm;
+  if (dsa_status st = make_tmap(&tm, latent, 2, 576, (uint64_t)B * kv_len, 64)) return st;
+  cudaError_t e = dsa::launch_latent_attn_dense(tm, a, idx, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "latent_attn_dense launch");
+  return DSA_OK;
+}
+
+dsa_status dsa_mass_coverage(int rows, int H, const float* lse_sparse, const float* lse_dense, float* m_out,
+                             float* per_head_out, float* min_out, void* stream) {
+  DSA_CHECK(rows >= 0 && H >= 1, DSA_ERR_INVALID_ARG, "need rows >= 0 and H >= 1");
+  DSA_CHECK(lse_sparse && lse_dense, DSA_ERR_INVALID_ARG, "null tensor pointer");
+  cudaError_t e = dsa::launch_mass_coverage(rows, H, lse_sparse, lse_dense, m_out, per_head_out, min_out,
+                                            (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "mass_coverage launch");
+  return DSA_OK;
+}
+
 // ---------------------------------------------------------------- decode indexer
 static constexpr int kScanChunkTiles = 8;
 

@@ -80,6 +80,21 @@ struct AttnArgs {
   DeviceStatus* status;
 };
 
+// Attention over dense causal key tiles, masked to the selection
+// (latent_attn_dense.cu): 16 heads, latent rows 576 / value 512.
+struct DenseAttnArgs {
+  int B, nq, q_offset, kv_len, k;
+  int nblk;                    // 8-token blocks per sequence
+  int kv_tiles;                // 64-key tiles of a sequence's history (words per selection row)
+  float scale_log2;
+  const uint16_t* q;           // [B, nq, 16, 576] bf16
+  const uint64_t* sel_bits;    // [B, nq, kv_tiles] or null (every causal key)
+  uint16_t* out;               // [B, nq, 16, 512] bf16
+  float* lse;                  // [B, nq, 16] or null
+  DeviceStatus* status;
+  uint64_t timeout_ns;
+};
+
 // Sparse-stage indexer KL on the selected set, forward and backward (indexer_kl.cu).
 constexpr int kMaxKLTopk = 4096;
 struct KLArgs {
@@ -127,6 +142,11 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, int grid, cudaStream_t stream)
 // H = 128, Dqk = 576, Dv = 512; one 2-CTA cluster per sequence (a.rows).
 cudaError_t launch_latent_attn_decode(const AttnArgs& a, cudaStream_t stream);
 size_t latent_attn_decode_smem();
+cudaError_t launch_latent_attn_dense(const CUtensorMap& tmap_lat, const DenseAttnArgs& a, const int32_t* idx,
+                                     cudaStream_t stream);
+size_t latent_attn_dense_smem();
+cudaError_t launch_mass_coverage(int rows, int H, const float* lse_sparse, const float* lse_dense, float* m_out,
+                                 float* per_head_out, float* min_out, cudaStream_t stream);
 size_t indexer_kl_smem_bytes(int dI, int k);
 size_t attn_teacher_smem_bytes(int k);
 cudaError_t launch_attn_teacher(const TeacherArgs& a, cudaStream_t stream);

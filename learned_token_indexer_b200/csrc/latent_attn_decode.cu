@@ -41,6 +41,7 @@
 #include <cuda_bf16.h>
 
 #include "kernels.h"
+#include "latent_attn.cuh"
 #include "sm100.cuh"
 
 namespace dsa {
@@ -162,34 +163,16 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   return s;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-template <int N>
-__device__ __forceinline__ void regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xffff0000u); }
-
-// Offset of 16-byte chunk `ch` (0..7) of row `n` in a 64-row block of the
-// 128-byte swizzled layout.
-__device__ __forceinline__ uint32_t swz_off(uint32_t n, uint32_t ch) {
-  return (n >> 3) * 1024u + (n & 7u) * 128u + ((ch ^ (n & 7u)) << 4);
-}
+using lattn::pack_bf16x2;
+using lattn::regs_dec;
+using lattn::regs_inc;
+using lattn::swz_off;
 
 }  // namespace
 
@@ -386,8 +369,10 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_decode_kernel(const A
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const float2 z = ffma2(make_float2(s[2 * j], s[2 * j + 1]), make_float2(1.0f, 1.0f), make_float2(-msub, -msub));
-        p[j] = pack_bf16x2(ex2_approx(z.x), ex2_approx(z.y));
-        lsum = ffma2(make_float2(bf16_lo(p[j]), bf16_hi(p[j])), make_float2(1.0f, 1.0f), lsum);
+        const float2 e = make_float2(ex2_approx(z.x), ex2_approx(z.y));
+        p[j] = pack_bf16x2(e.x, e.y);
+        // the denominator sums the unrounded probabilities (its log is the lse)
+        lsum = ffma2(e, make_float2(1.0f, 1.0f), lsum);
       }
       l_run = l_run * alpha + (lsum.x + lsum.y);
       // P of tile i goes to pbuf[i % 2]: P V of tile i - 2 must have read it.
