@@ -82,6 +82,8 @@ def kernel_source_hash(files):
 KERNEL_SOURCES = {
     "indexer_topk_prefill": ["indexer_topk_prefill.cu", "indexer_common.cuh", "select.cuh", "sm100.cuh"],
     "sparse_attn": ["sparse_attn.cu", "sm100.cuh"],
+    "dense_attn": ["latent_attn_dense.cu", "latent_attn.cuh", "sm100.cuh"],
+    "latent_attn_decode": ["latent_attn_decode.cu", "latent_attn.cuh", "sm100.cuh"],
     "indexer_scan": ["indexer_scan.cu", "indexer_common.cuh", "sm100.cuh"],
     "topk_rows": ["topk.cu", "select.cuh"],
     "indexer_kl": ["indexer_kl.cu", "sm100.cuh"],
@@ -188,6 +190,12 @@ class PrefillRun:
         if w.fp8:
             self.kw = dict(q_scale=self.d["q_scale"], k_scale=self.d["k_scale"])
         self.launches_per_step = 0
+        # the attention path the library's length dispatch takes (§2); every
+        # chunk of these workloads takes the same one
+        paths = {dsa.prefill_attention_path(w.B, min(w.n, c0 + self.chunk) - c0, c0, w.n, w.H, w.Dqk, w.Dv, w.k)
+                 for c0 in range(0, w.n, self.chunk)}
+        assert len(paths) == 1, "mixed attention paths within one workload"
+        self.attn_name = "dense_attn" if paths.pop() == dsa.PATH_DENSE_MASKED else "sparse_attn"
 
     def step(self, ev=None):
         dsa, w, d = self.dsa, self.w, self.d
@@ -202,14 +210,15 @@ class PrefillRun:
             dsa.indexer_topk_prefill(d["qI"][sl], d["kI"], d["w"][sl], w.k, q_offset=c0, idx_out=self.idx[sl],
                                      workspace=self.ws_idx, **kw)
             e1 = self._rec(ev)
-            dsa.sparse_attn_prefill(d["q"][sl], d["latent"], self.idx[sl], w.Dv, scale=w.scale, out=self.out[sl],
-                                    workspace=self.ws_att)
+            dsa.attn_prefill(d["q"][sl], d["latent"], self.idx[sl], w.Dv, q_offset=c0, scale=w.scale,
+                             out=self.out[sl], workspace=self.ws_att)
             e2 = self._rec(ev)
             if ev is not None:
                 ev["indexer_topk_prefill"].append((e0, e1))
-                ev["sparse_attn"].append((e1, e2))
+                ev[self.attn_name].append((e1, e2))
             triv = c0 < w.k
-            launches += 2 + (1 if triv else 0)
+            # indexer (+ trivial rows), attention (+ memset and selection bits on the dense path)
+            launches += 2 + (1 if triv else 0) + (2 if self.attn_name == "dense_attn" else 0)
         self.launches_per_step = launches
 
     @staticmethod
@@ -249,10 +258,46 @@ class PrefillRun:
                                       "rows": int(rec.numel()),
                                       "definition": "|T ∩ S| / |T|, T = bf16 selection of the same draws, "
                                                     "S = e4m3 selection; rows with t + 1 > k"}}
-        out["recall_by_margin"] = self._recall_by_margin(rec_all, ws)
+        mass = self._mass_coverage(ref, ws)
+        out["mass_coverage"] = mass["summary"]
+        out["recall_by_margin"] = self._recall_by_margin(rec_all, ws, mass_loss=mass["loss"])
         return out
 
-    def _recall_by_margin(self, rec_all, ws, strip: int = 512, buckets: int = 4):
+    def _mass_coverage(self, ref, ws):
+        """Teacher mass coverage M_k (eq. (15)) of both selections: the dense
+        causal attention's probabilities (heads summed, L1-normalised, eq.
+        (16)) on the selected positions, from the lse of the dense attention
+        and of the sparse attention over each selection (dsa_mass_coverage).
+        §2 asks FP8 validation to compare set overlap and this coverage."""
+        w, d, dsa = self.w, self.d, self.dsa
+        scratch = torch.empty_like(self.out)
+        _, lse_d = dsa.attn_dense_prefill(d["q"], d["latent"], w.Dv, scale=w.scale, out=scratch, return_lse=True,
+                                          workspace=ws)
+        res = {}
+        for name, sel in (("e4m3", self.idx), ("bf16", ref)):
+            _, lse_s = dsa.sparse_attn_prefill(d["q"], d["latent"], sel, w.Dv, scale=w.scale, out=scratch,
+                                               return_lse=True, workspace=ws)
+            res[name] = dsa.mass_coverage(lse_s, lse_d)
+        torch.cuda.synchronize()
+        ws.check()
+        summary = {}
+        for name, (m, mn) in res.items():
+            mm, mh = m[:, w.k:].flatten().double(), mn[:, w.k:].flatten().double()
+            qs = torch.quantile(mm, torch.tensor([0.01, 0.5], dtype=torch.float64, device=mm.device))
+            summary[name] = {"mean": round(float(mm.mean()), 5), "p01": round(float(qs[0]), 5),
+                             "median": round(float(qs[1]), 5), "min": round(float(mm.min()), 5),
+                             "lowest_head_mean": round(float(mh.mean()), 5), "lowest_head_min": round(float(mh.min()), 5)}
+        loss_all = (res["bf16"][0] - res["e4m3"][0]).double()
+        loss = loss_all[:, w.k:].flatten()
+        summary["loss_bf16_minus_e4m3"] = {"mean": float(loss.mean()), "max": float(loss.max()),
+                                           "min": float(loss.min())}
+        summary["definition"] = ("M_k = sum over the selection of the dense attention probability (eq. (15)), "
+                                 "teacher = heads summed then L1-normalised (eq. (16)); lowest_head = the "
+                                 "smallest per-head coverage; rows with t + 1 > k; bf16 = the selection of "
+                                 "the same draws rounded to bf16, e4m3 = the timed FP8 selection")
+        return {"summary": summary, "loss": loss_all}
+
+    def _recall_by_margin(self, rec_all, ws, strip: int = 512, buckets: int = 4, mass_loss=None):
         """Recall of the e4m3 selection grouped by the bf16 cut-off margin
         Delta_k = s_(k) - s_(k+1) (eq. (18), §3.1: small margins are where a
         perturbation swaps boundary tokens).  On the last `strip` rows of the
@@ -277,10 +322,14 @@ class PrefillRun:
             m = (margin >= lo) & ((margin <= hi) if i == buckets - 1 else (margin < hi))
             if int(m.sum()) == 0:
                 continue
-            rows.append({"margin": [round(lo, 6), round(hi, 6)], "rows": int(m.sum()),
-                         "mean_recall": round(float(rec[m].mean()), 5)})
+            row = {"margin": [round(lo, 6), round(hi, 6)], "rows": int(m.sum()),
+                   "mean_recall": round(float(rec[m].mean()), 5)}
+            if mass_loss is not None:
+                row["mean_mass_loss"] = float(mass_loss[0, t0:][m].mean())
+            rows.append(row)
         return {"strip": f"rows {t0}..{w.n - 1} of sequence 0", "buckets": rows,
-                "definition": "Delta_k = s_(k) - s_(k+1) of the bf16 scores (eq. (18)); quartile buckets"}
+                "definition": "Delta_k = s_(k) - s_(k+1) of the bf16 scores (eq. (18)); quartile buckets; "
+                              "mass loss = M_k(bf16 selection) - M_k(e4m3 selection)"}
 
     def kernel_work(self):
         w = self.w
@@ -294,13 +343,25 @@ class PrefillRun:
             "indexer_topk_prefill": {"flops": 2 * w.HI * w.dI * w.B * pairs, "unit": "TFLOP/s",
                                      "per_unit": f"2*HI*dI = {2 * w.HI * w.dI} FLOP per scored (t,s) pair",
                                      "units": w.B * pairs},
-            "sparse_attn": {"flops": 2 * w.H * w.B * ent * (w.Dqk + w.Dv), "unit": "TFLOP/s",
-                            "per_unit": f"2*H*(Dqk+Dv) = {2 * w.H * (w.Dqk + w.Dv)} FLOP per selected entry",
-                            "units": w.B * ent, "gather_bytes": w.B * ent * w.Dqk * 2},
+            self.attn_name: self._attn_work(ent),
         }
 
+    def _attn_work(self, ent):
+        w = self.w
+        r = {"flops": 2 * w.H * w.B * ent * (w.Dqk + w.Dv), "unit": "TFLOP/s",
+             "per_unit": f"2*H*(Dqk+Dv) = {2 * w.H * (w.Dqk + w.Dv)} FLOP per selected entry",
+             "units": w.B * ent}
+        if self.attn_name == "sparse_attn":
+            r["gather_bytes"] = w.B * ent * w.Dqk * 2
+        else:
+            pairs = sum(t + 1 for t in range(w.n))
+            r["path"] = ("dense masked (short prefill, §2): every causal key tile is multiplied, "
+                         f"{2 * w.H * w.B * pairs * (w.Dqk + w.Dv) / 1e12:.3f} TFLOP per step executed")
+        return r
+
     def host_inputs(self):
-        return {k: v.cpu().pin_memory() for k, v in self.d.items() if isinstance(v, torch.Tensor)}
+        return {k: v.cpu().pin_memory() for k, v in self.d.items()
+                if isinstance(v, torch.Tensor) and not k.endswith("_bf16")}
 
     def load_inputs(self, host):
         for k, v in host.items():
@@ -782,7 +843,7 @@ def measure_workload(w, args, dev, world, rank, local, steps, warmup, cpu_budget
             peak = peaks["hbm_gbs"]
             ach = per_launch / (t_launch * 1e-3) / 1e9
             bound = "hbm"
-        tkey = {"indexer_topk_decode": "indexer_scan", "sparse_attn_decode": "sparse_attn"}.get(name, name)
+        tkey = {"indexer_topk_decode": "indexer_scan", "sparse_attn_decode": "latent_attn_decode"}.get(name, name)
         # the training step's selection and attention are the prefill workload's launches
         twl = "prefill" if (w.kind == "train" and name in ("indexer_topk_prefill", "sparse_attn")) else w.name
         kernels[name] = {"bound": bound, "achieved": round(ach, 2), "peak": peak, "unit": wk["unit"],
@@ -827,7 +888,7 @@ def measure_workload(w, args, dev, world, rank, local, steps, warmup, cpu_budget
 # The default run: the largest single-GPU prefill configuration is the line's
 # value; the other configurations of the metric are sub-records.
 DEFAULT_WORKLOAD = "long_prefill"
-DEFAULT_SUBS = ("prefill", "prefill_fp8", "decode")
+DEFAULT_SUBS = ("prefill", "prefill_fp8", "decode", "short_prefill")
 BASELINE_METRIC = "prefill query-tokens/s (indexer+top-k+sparse attn) & decode tokens/s; % roofline"
 
 

@@ -153,6 +153,23 @@ dsa_status dsa_attn_dense_prefill(int B, int nq, int q_offset, int kv_len, int H
                                   const void* q, const void* latent, const int32_t* idx, void* out, float* lse,
                                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* Length dispatch of the prefill attention (§2: the serving side picks the
+ * path by length; masked dense attention wins for short histories).
+ * dsa_prefill_attention_path returns DSA_PATH_DENSE_MASKED when the chunk's
+ * longest history (q_offset + nq keys) is at most 4096 and the shape is the
+ * dense kernel's (H = 16, Dqk = 576, Dv = 512), else DSA_PATH_GATHER (the
+ * threshold is where the two paths' measured times cross on one B200 with
+ * k = 2048).  dsa_attn_prefill runs eq. (3) on that path with the arguments
+ * of dsa_attn_dense_prefill (idx required); both paths give the same result
+ * on the same selection.  Its workspace is dsa_attn_prefill_workspace(...)
+ * bytes. */
+enum { DSA_PATH_GATHER = 0, DSA_PATH_DENSE_MASKED = 1 };
+int dsa_prefill_attention_path(int B, int nq, int q_offset, int kv_len, int H, int Dqk, int Dv, int k);
+size_t dsa_attn_prefill_workspace(int B, int nq, int q_offset, int kv_len, int H, int Dqk, int Dv, int k);
+dsa_status dsa_attn_prefill(int B, int nq, int q_offset, int kv_len, int H, int Dqk, int Dv, int k, float scale,
+                            const void* q, const void* latent, const int32_t* idx, void* out, float* lse,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
 /* Teacher mass coverage of a selection (§3.1, eq. (15)): for each of `rows`
  * query rows and each head h, the dense attention probabilities on the
  * selected positions sum to exp(lse_sparse[r, h] - lse_dense[r, h]) (the lse

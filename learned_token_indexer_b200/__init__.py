@@ -193,6 +193,36 @@ def attn_dense_prefill(q, latent, dv: int, idx=None, k: Optional[int] = None, q_
     return (out, lse) if lse is not None else out
 
 
+PATH_GATHER, PATH_DENSE_MASKED = 0, 1
+
+
+def prefill_attention_path(B: int, nq: int, q_offset: int, kv_len: int, H: int, Dqk: int, Dv: int, k: int) -> int:
+    """The prefill attention path the library picks for a chunk (§2 length
+    dispatch): PATH_DENSE_MASKED for short histories, else PATH_GATHER."""
+    return int(lib().dsa_prefill_attention_path(B, nq, q_offset, kv_len, H, Dqk, Dv, k))
+
+
+def attn_prefill(q, latent, idx, dv: int, q_offset: int = 0, scale: Optional[float] = None, out=None, lse=None,
+                 return_lse: bool = False, workspace: Optional[Workspace] = None):
+    """Eq. (3) for a prefill chunk on the path the length dispatch picks (the
+    dense masked path for short histories, the gathering path otherwise);
+    arguments as attn_dense_prefill with a required index tensor."""
+    B, nq, H, Dqk = q.shape
+    kv_len = latent.shape[1]
+    k = idx.shape[-1]
+    scale = Dqk ** -0.5 if scale is None else scale
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, nq, H, dv), dtype=torch.bfloat16, device=dev)
+    if return_lse and lse is None:
+        lse = torch.empty((B, nq, H), dtype=torch.float32, device=dev)
+    L = lib()
+    wsb = _ws(workspace, dev).get(L.dsa_attn_prefill_workspace(B, nq, q_offset, kv_len, H, Dqk, dv, k))
+    _check(L.dsa_attn_prefill(B, nq, q_offset, kv_len, H, Dqk, dv, k, float(scale), _ptr(q), _ptr(latent),
+                              _ptr(idx), _ptr(out), _ptr(lse), _ptr(wsb), wsb.numel(), _stream(dev)))
+    return (out, lse) if lse is not None else out
+
+
 def mass_coverage(lse_sparse, lse_dense, per_head: bool = False):
     """Teacher mass coverage M_k of eq. (15) per query row from the two lse
     tensors [..., H]: returns (M, min over heads) [...] (and the per-head

@@ -35,6 +35,9 @@ SIGNATURES = {
     "dsa_attn_dense_prefill_workspace": (_sz, [_i, _i, _i, _i]),
     "dsa_attn_dense_prefill": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "dsa_mass_coverage": (_i, [_i, _i, _p, _p, _p, _p, _p, _p]),
+    "dsa_prefill_attention_path": (_i, [_i, _i, _i, _i, _i, _i, _i, _i]),
+    "dsa_attn_prefill_workspace": (_sz, [_i, _i, _i, _i, _i, _i, _i, _i]),
+    "dsa_attn_prefill": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "dsa_attn_teacher_prefill": (_i, [_i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "dsa_indexer_kl_sparse": (_i, [_i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _f, _p, _p, _p, _p, _p, _p, _sz, _p]),
 }

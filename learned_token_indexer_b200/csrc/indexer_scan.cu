@@ -340,7 +340,7 @@ static cudaError_t launch_scan_t(const CUtensorMap& tq, const CUtensorMap& tk, c
                                  cudaStream_t stream) {
   const size_t smem = scan_smem_bytes<HI, FP8, KB>();
   auto kern = indexer_scan_kernel<HI, FP8, KB>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = setup_once_per_device([&]() { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); });
   if (e != cudaSuccess) return e;
   kern<<<grid, kScanThreads, smem, stream>>>(tq, tk, a);
   return cudaGetLastError();

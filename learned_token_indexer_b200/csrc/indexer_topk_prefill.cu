@@ -541,7 +541,7 @@ static cudaError_t launch_prefill_t(const CUtensorMap& tq, const CUtensorMap& tk
                                     cudaStream_t stream) {
   using C = PrefillConfig<HI, FP8, KB>;
   auto kern = indexer_topk_prefill_kernel<HI, FP8, KB, C::STAGES>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  cudaError_t e = setup_once_per_device([&]() { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem); });
   if (e != cudaSuccess) return e;
   kern<<<grid, kPrefillThreads, C::kSmem, stream>>>(tq, tk, a);
   return cudaGetLastError();

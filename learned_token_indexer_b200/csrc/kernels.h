@@ -1,12 +1,36 @@
 // kernels.h -- internal interface between the C ABI (api.cu) and the kernels.
 #pragma once
 #include <cstdint>
+#include <mutex>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace dsa {
 
 struct DeviceStatus;
+
+// A kernel's one-time host set-up (its shared-memory attribute, checks of its
+// compiled register count): `setup` runs on the first launch from a call site
+// on each device and its result is reused, keeping host calls off the launch
+// path.  Thread-safe.
+template <typename F>
+cudaError_t setup_once_per_device(F&& setup) {
+  constexpr int kMaxDev = 64;
+  static std::mutex mu;
+  static bool done[kMaxDev] = {};
+  static cudaError_t result[kMaxDev] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return setup();
+  std::lock_guard<std::mutex> lock(mu);
+  if (!done[dev]) {
+    result[dev] = setup();
+    done[dev] = true;
+  }
+  return result[dev];
+}
 
 // Dense score rows (indexer_scan.cu).
 constexpr int kScanMaxBalancedRows = 4096;

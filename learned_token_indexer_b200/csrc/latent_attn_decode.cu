@@ -603,12 +603,14 @@ size_t latent_attn_decode_smem() { return smem_bytes(); }
 cudaError_t launch_latent_attn_decode(const AttnArgs& a, cudaStream_t stream) {
   // the warpgroups' register budgets add up to the launch allocation; a
   // build that allocated differently would make the increase wait forever
-  cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, latent_attn_decode_kernel);
-  if (e != cudaSuccess) return e;
-  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   const size_t smem = smem_bytes();
-  e = cudaFuncSetAttribute(latent_attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = setup_once_per_device([smem]() {
+    cudaFuncAttributes fa;
+    cudaError_t r = cudaFuncGetAttributes(&fa, latent_attn_decode_kernel);
+    if (r != cudaSuccess) return r;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    return cudaFuncSetAttribute(latent_attn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  });
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2u * (unsigned)a.rows, 1, 1);

@@ -528,8 +528,9 @@ cudaError_t launch_latent_attn_dense(const CUtensorMap& tmap_lat, const DenseAtt
     if (e != cudaSuccess) return e;
   }
   const size_t smem = smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(latent_attn_dense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  cudaError_t e = setup_once_per_device([smem]() {
+    return cudaFuncSetAttribute(latent_attn_dense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  });
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2u * (unsigned)(a.B * a.nblk), 1, 1);

@@ -674,12 +674,14 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, int grid, cudaStream_t stream)
     return cudaErrorInvalidValue;
   // the warpgroups' register budgets add up to the launch allocation; a
   // build that allocated differently would make the increase wait forever
-  cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, sparse_attn_kernel);
-  if (e != cudaSuccess) return e;
-  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   const size_t smem = attn_smem();
-  e = cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = setup_once_per_device([smem]() {
+    cudaFuncAttributes fa;
+    cudaError_t r = cudaFuncGetAttributes(&fa, sparse_attn_kernel);
+    if (r != cudaSuccess) return r;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    return cudaFuncSetAttribute(sparse_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  });
   if (e != cudaSuccess) return e;
   sparse_attn_kernel<<<grid, kThreads, smem, stream>>>(a);
   return cudaGetLastError();

@@ -68,12 +68,16 @@ DECODE_FP8 = Workload("decode_fp8", "decode", B=64, n=0, HI=64, dI=128, k=2048, 
                       qk_dist="normal", w_std=0.1, fp8=True, seed=3, L_min=4096, L_max=65536)
 LONG = Workload("long_prefill", "prefill", B=1, n=131072, HI=64, dI=128, k=2048, H=16, Dqk=576,
                 Dv=512, qk_dist="normal", w_std=0.1, chunk=8192, seed=4)
+# Short prefill (every row has t + 1 <= k): the case §2 says DSA runs as
+# masked dense attention; the prefill workload's distributions, 8 sequences.
+SHORT_PREFILL = Workload("short_prefill", "prefill", B=8, n=2048, HI=64, dI=128, k=2048, H=16, Dqk=576, Dv=512,
+                         qk_dist="int", qk_int_max=3, w_den=16, seed=5)
 # Sparse training stage (eq. (8)): the prefill workload's inputs; the teacher
 # comes from the sparse attention on each row's selected set.
 INDEXER_KL = Workload("indexer_kl", "train", B=1, n=8192, HI=64, dI=128, k=2048, H=16, Dqk=576, Dv=512,
                       qk_dist="int", qk_int_max=3, w_den=16, seed=1)
 
-ALL = {w.name: w for w in (TINY, PREFILL, PREFILL_FP8, DECODE, DECODE_FP8, LONG, INDEXER_KL)}
+ALL = {w.name: w for w in (TINY, PREFILL, PREFILL_FP8, DECODE, DECODE_FP8, LONG, SHORT_PREFILL, INDEXER_KL)}
 
 
 def scaled(w: Workload, **changes) -> Workload:

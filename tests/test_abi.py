@@ -151,3 +151,31 @@ def test_attn_teacher_argument_checks(lib):
     assert call(scale=float("nan")) == 1
     assert call(wsb=8) == 3
     assert call(nq=0) == 0
+
+
+def test_prefill_attention_length_dispatch(lib):
+    """§2: short histories take the masked dense path, long ones gather; only
+    the dense kernel's shape (16 heads, 576/512 latent rows) can go dense."""
+    path = lib.dsa_prefill_attention_path
+    assert path(1, 2048, 0, 2048, 16, 576, 512, 2048) == dsa.PATH_DENSE_MASKED
+    assert path(4, 4096, 0, 4096, 16, 576, 512, 2048) == dsa.PATH_DENSE_MASKED
+    assert path(1, 8192, 0, 8192, 16, 576, 512, 2048) == dsa.PATH_GATHER
+    assert path(1, 1024, 3584, 8192, 16, 576, 512, 2048) == dsa.PATH_GATHER    # chunk ends past 4096
+    assert path(1, 512, 0, 512, 4, 64, 64, 16) == dsa.PATH_GATHER              # other head / width
+    assert path(1, 0, 0, 16, 16, 576, 512, 16) == dsa.PATH_GATHER
+    assert lib.dsa_attn_prefill_workspace(1, 2048, 0, 2048, 16, 576, 512, 2048) >= 256 + 2048 * 32 * 8
+    assert lib.dsa_attn_prefill_workspace(1, 8192, 0, 8192, 16, 576, 512, 2048) == lib.dsa_sparse_attn_workspace()
+
+
+def test_dense_attention_host_checks(lib):
+    ws = (C.c_uint8 * 512)()
+    wsp = C.cast(ws, C.c_void_p)
+    fake = C.c_void_p(4096)          # never dereferenced: the checks fail first
+    st = lib.dsa_attn_dense_prefill(1, 16, 0, 16, 8, 576, 512, 16, 0.1, fake, fake, None, fake, None, wsp, 512, None)
+    assert st == 2                   # DSA_ERR_UNSUPPORTED (8 heads)
+    st = lib.dsa_attn_dense_prefill(1, 16, 8, 16, 16, 576, 512, 16, 0.1, fake, fake, None, fake, None, wsp, 512, None)
+    assert st == 1                   # q_offset + nq > kv_len
+    st = lib.dsa_attn_dense_prefill(1, 16, 0, 16, 16, 576, 512, 16, 0.1, fake, fake, fake, fake, None, wsp, 16, None)
+    assert st == 3                   # workspace too small for the selection bits
+    st = lib.dsa_mass_coverage(4, 0, fake, fake, None, None, None, None)
+    assert st == 1

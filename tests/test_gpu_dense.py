@@ -165,3 +165,24 @@ def test_dense_masked_full_prefill_sampled():
     torch.cuda.synchronize()
     _no_device_errors(ws)
     _check_rows(d["q"], d["latent"], idx, out, lse, 0, W.sample_rows(w, 256), w.scale)
+
+
+def test_attn_prefill_length_dispatch_gives_the_same_result():
+    """dsa_attn_prefill picks the dense masked path for a short history and
+    the gathering path for a long one; on the same selection both equal the
+    gathering kernel's output within the attention tolerance."""
+    ws = dsa.Workspace("cuda")
+    for kv, q0, nq, k in ((1000, 0, 1000, 128), (4300, 4150, 150, 96)):
+        qall, lat = _inputs(1, kv, kv, 11 + kv)
+        q = qall[:, q0:q0 + nq].contiguous()
+        idx = W.make_selection(1, nq, kv, k, q_offset=q0, seed=kv, device="cuda")
+        path = dsa.prefill_attention_path(1, nq, q0, kv, 16, 576, 512, k)
+        assert path == (dsa.PATH_DENSE_MASKED if kv <= 4096 else dsa.PATH_GATHER)
+        out, lse = dsa.attn_prefill(q, lat, idx, 512, q_offset=q0, scale=1 / 24, return_lse=True, workspace=ws)
+        ref, ref_lse = dsa.sparse_attn_prefill(q, lat, idx, 512, scale=1 / 24, return_lse=True, workspace=ws)
+        torch.cuda.synchronize()
+        _no_device_errors(ws)
+        diff = (out.float() - ref.float()).abs() - (ATOL + RTOL * ref.float().abs())
+        assert float(diff.max()) <= 0.0
+        assert float((lse - ref_lse).abs().max()) <= 2e-3
+        _check_rows(q, lat, idx, out, lse, q0, [(0, i) for i in range(0, nq, 13)])
