@@ -12,8 +12,9 @@
 //   [512 + 32r, 512 + 32r + 32) of each selected row and of the queries.
 //   Per tile of 64 selected rows it forms the partial logits over its own
 //   columns, S_r = Q_r C_r^T (M 128 x N 64, K 288), sends them to the other
-//   CTA (st.async into its shared memory, counted by the receiver's mbarrier)
-//   and adds the partial it receives, so both CTAs hold the same full logits
+//   CTA (one 16 KB TMA bulk copy per warpgroup from a local staging buffer,
+//   counted by the receiver's mbarrier) and adds the partial it receives,
+//   so both CTAs hold the same full logits
 //   S = S_0 + S_1 (the same fp32 sum on both sides), take the same softmax
 //   decisions, and accumulate O_r += P C_r[:, value]  (M 128 x N 256, K 64)
 //   for their own half of the value columns.  No row is gathered twice and no
@@ -33,9 +34,8 @@
 // warpgroup owns head h = TMEM lane h); 8 issues the logits MMAs and owns
 // TMEM; 9 issues P V; 10 issues the bulk copies; 11 the rope copies and the
 // slot mask; 12-19 convert staged rows.  Registers move to the softmax warps
-// with setmaxnreg.  The queries live in TMEM (A operand of the logits); P is
-// written to one of two shared-memory buffers (A operand of P V), so the
-// softmax of tile i + 1 overlaps P V of tile i.  Online softmax in base 2
+// with setmaxnreg.  The queries and P live in TMEM (the A operands of the
+// logits and of P V).  Online softmax in base 2
 // with a lazy reference maximum: O and l are rescaled only when a tile's
 // maximum exceeds the reference by more than 2^8.
 #include <cuda_bf16.h>
@@ -57,10 +57,9 @@ constexpr int kSlotBytes = kTile * 128;                  // one 64-column block 
 constexpr int kSwzBytes = 5 * kSlotBytes;                // 4 value blocks + the rope block
 constexpr int kRowBytes = 512;                           // a row's value half for this CTA
 constexpr int kRawBytes = kTile * kRowBytes;
-constexpr int kPBytes = kHeads * kTile * 2;              // P of one tile, bf16, 128-byte swizzled rows
-constexpr int kXPitch = 272;                             // 64 fp32 + 16 B: one head's partial logits
-constexpr int kXBytes = kHeads * kXPitch;
-constexpr uint32_t kXTx = kHeads * kTile * 4;            // bytes the other CTA sends per tile
+constexpr int kXHalf = kHeads * 32 * 4;                  // one warpgroup's partial logits (16 KB)
+constexpr int kXBytes = 2 * kXHalf;
+constexpr uint32_t kXTx = kXBytes;                       // bytes the other CTA sends per tile
 constexpr int kSoftWarps = 8;
 constexpr int kMmaWarp = 8;                               // logits issuer, TMEM owner
 constexpr int kPvWarp = 9;                                // P V issuer
@@ -78,22 +77,24 @@ constexpr int kLaunchRegs = 96;
 constexpr int kRegsSoft = 168, kRegsOther = 48;
 static_assert(2 * kRegsSoft + 3 * kRegsOther == 5 * kLaunchRegs, "register split must match the launch");
 constexpr uint32_t kBarSoft = 2;                          // named barrier of the softmax warps
+constexpr uint32_t kBarHalf0 = 3;                         // + g: the softmax warps of warpgroup g
 
 // TMEM columns (512 allocated)
 constexpr uint32_t kTmemO = 0;       // 256 fp32: O for this CTA's value columns
 constexpr uint32_t kTmemQ = 256;     // 144: queries, bf16 pairs (128 value + 16 rope)
+constexpr uint32_t kTmemP = 416;     // 32: P, bf16 pairs (A operand of P V)
 constexpr uint32_t kTmemS = 448;     // 64 fp32: partial logits
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kIdescS = instr_desc(1u, 128u, 64u);          // K-major x K-major, M 128, N 64
-constexpr uint32_t kIdescPV = instr_desc_bf16_bmn(128u, 256u);   // A K-major, B MN-major, M 128, N 256
+constexpr uint32_t kIdescPV = instr_desc_bf16_bmn(128u, 256u);   // A (TMEM), B MN-major, M 128, N 256
 constexpr float kRescaleThreshold = 8.0f;                         // log2 units
 
 struct Smem {
   uint8_t* swz;        // kSwz x kSwzBytes, 1024-aligned
-  uint8_t* pbuf;       // 2 x kPBytes: P of tiles i % 2
   uint8_t* raw;        // kRaw x kRawBytes: value halves, one 512-byte row per slot
-  uint8_t* x;          // kXBytes: the other CTA's partial logits, one row per head
+  uint8_t* x;          // kXBytes: the other CTA's partial logits (two 16 KB warpgroup halves)
+  uint8_t* xs;         // kXBytes: this CTA's partial logits, staged for the copy
   float* tmax;         // 2 x 2 x kHeads: each warpgroup's tile maximum per head (by tile parity)
   float* lsum;         // kHeads: warpgroup 1's softmax denominator at the end
   uint32_t* mask;      // kSwz x 2: valid slots of the tile
@@ -103,8 +104,8 @@ struct Smem {
   uint64_t* raw_empty; // kRaw: converted
   uint64_t* s_full;
   uint64_t* s_empty;
-  uint64_t* p_full;    // 2: P of tile i is in pbuf[i % 2]
-  uint64_t* o_done;    // 2: P V of tile i (committed to o_done[i % 2]) is done
+  uint64_t* p_full;    // P of the tile is in TMEM
+  uint64_t* o_done;    // P V of the tile is done
   uint64_t* x_full;    // the other CTA's partial for the tile is in x
   uint64_t* x_empty;   // the other CTA has read what this CTA wrote into it
   uint64_t* drain;     // 2: every MMA of the logits / P V issuer is done
@@ -116,7 +117,7 @@ struct Smem {
 constexpr int kNumBars = 2 * kSwz + 2 * kRaw + 2 + 2 + 2 + 2 + 2;
 
 __host__ __device__ constexpr size_t smem_bytes() {
-  return 1024 + (size_t)kSwz * kSwzBytes + 2 * kPBytes + (size_t)kRaw * kRawBytes + kXBytes + 5 * kHeads * 4 +
+  return 1024 + (size_t)kSwz * kSwzBytes + (size_t)kRaw * kRawBytes + 2 * kXBytes + 5 * kHeads * 4 +
          kSwz * 8 + kNumBars * 8 + 64;
 }
 
@@ -125,11 +126,11 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   uint8_t* p = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   s.swz = p;
   p += kSwz * kSwzBytes;
-  s.pbuf = p;
-  p += 2 * kPBytes;
   s.raw = p;
   p += kRaw * kRawBytes;
   s.x = p;
+  p += kXBytes;
+  s.xs = p;
   p += kXBytes;
   s.tmax = reinterpret_cast<float*>(p);
   p += 4 * kHeads * 4;
@@ -148,10 +149,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   b += kRaw;
   s.s_full = b++;
   s.s_empty = b++;
-  s.p_full = b;
-  b += 2;
-  s.o_done = b;
-  b += 2;
+  s.p_full = b++;
+  s.o_done = b++;
   s.x_full = b++;
   s.x_empty = b++;
   s.drain = b;
@@ -198,11 +197,9 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_decode_kernel(const A
     }
     mbar_init(sm.s_full, 1);
     mbar_init(sm.s_empty, kSoftWarps);
-    for (int j = 0; j < 2; ++j) {
-      mbar_init(&sm.p_full[j], kSoftWarps);
-      mbar_init(&sm.o_done[j], 1);
-      mbar_init(&sm.drain[j], 1);
-    }
+    mbar_init(sm.p_full, kSoftWarps);
+    mbar_init(sm.o_done, 1);
+    for (int j = 0; j < 2; ++j) mbar_init(&sm.drain[j], 1);
     mbar_init(sm.x_full, 1);    // one local arrival (with the byte count) + the other CTA's bytes
     mbar_init(sm.x_empty, 1);   // one arrival from the other CTA per tile
     *sm.last_valid = -1;
@@ -280,10 +277,13 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_decode_kernel(const A
     const uint32_t g = warp >> 2;                 // key half of the tile / value quarter of the output
     const uint32_t h = tid & 127u;                // head = TMEM lane
     const uint32_t lrow = (warp & 3u) * 32u;
-    const uint32_t x_off = h * kXPitch + g * 128u;
-    const uint32_t x_peer = map_to_cta(smem_u32(sm.x + x_off), peer);
+    // row h of a warpgroup's 16 KB block of partial logits: 128 bytes, its
+    // 16-byte chunks XOR-swizzled by h so that 8 rows cover every bank
+    const uint32_t x_row = g * (uint32_t)kXHalf + h * 128u;
+    const uint32_t x_peer = map_to_cta(smem_u32(sm.x + g * kXHalf), peer);
     const uint32_t xfull_peer = map_to_cta(smem_u32(sm.x_full), peer);
     const uint32_t xempty_peer = map_to_cta(smem_u32(sm.x_empty), peer);
+    const bool leader = (tid & 127u) == 0u;       // issues its warpgroup's copy
     const float c = a.scale_log2;
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
@@ -307,18 +307,30 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_decode_kernel(const A
       if (lane == 0) mbar_arrive(sm.s_empty);
       // exchange partial logits with the other CTA of the pair: wait until it
       // has read the previous tile's, then write this tile's into it
-      if (i >= 1) ok = ok && mbar_wait_cluster(sm.x_empty, (uint32_t)(i - 1) & 1u, ctl, 0x2402);
+      // (and this warpgroup's previous copy has read the staging buffer)
+      if (leader) {
+        if (i >= 1) ok = ok && mbar_wait_cluster(sm.x_empty, (uint32_t)(i - 1) & 1u, ctl, 0x2402);
+        bulk_wait_read_all();
+      }
+      named_bar_sync(kBarHalf0 + g, 128);
       if (ok) {
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          st_async_v4(x_peer + 16 * j, s[4 * j], s[4 * j + 1], s[4 * j + 2], s[4 * j + 3], xfull_peer);
+          *reinterpret_cast<float4*>(sm.xs + x_row + ((j ^ (h & 7u)) << 4)) =
+              make_float4(s[4 * j], s[4 * j + 1], s[4 * j + 2], s[4 * j + 3]);
+        fence_proxy_async_smem();
+      }
+      named_bar_sync(kBarHalf0 + g, 128);
+      if (leader && ok) {
+        bulk_s2cluster(x_peer, smem_u32(sm.xs + g * kXHalf), kXHalf, xfull_peer);
+        bulk_commit_group();
       }
       ok = ok && mbar_wait_cluster(sm.x_full, (uint32_t)i & 1u, ctl, 0x2403);
       if (ok) {
-        const float4* xr = reinterpret_cast<const float4*>(sm.x + x_off);
+        const uint8_t* xr = sm.x + x_row;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float4 v = xr[j];
+          const float4 v = *reinterpret_cast<const float4*>(xr + ((j ^ (h & 7u)) << 4));
           s[4 * j] += v.x;
           s[4 * j + 1] += v.y;
           s[4 * j + 2] += v.z;
@@ -351,8 +363,10 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_decode_kernel(const A
       float* tm = sm.tmax + ((uint32_t)i & 1u) * 2 * kHeads;
       tm[g * kHeads + h] = mt;
       named_bar_sync(kBarSoft, kSoftWarps * 32);
-      // every softmax thread has read x: the other CTA may write the next tile's
-      if (tid == 0) mbar_arrive_cluster(xempty_peer);
+      // every softmax thread has read x: the other CTA may write the next
+      // tile's (signalled by a thread that issues no bulk copy: a
+      // cluster-scope release by the copy's issuer would wait for the copy)
+      if (tid == 96) mbar_arrive_cluster(xempty_peer);
       mt = fmaxf(mt, tm[(g ^ 1u) * kHeads + h]);
       float alpha = 1.0f;
       bool rescale = false;
@@ -375,17 +389,12 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_decode_kernel(const A
         lsum = ffma2(e, make_float2(1.0f, 1.0f), lsum);
       }
       l_run = l_run * alpha + (lsum.x + lsum.y);
-      // P of tile i goes to pbuf[i % 2]: P V of tile i - 2 must have read it.
-      // A rescale also needs P V of tile i - 1 folded into O first.
-      const uint32_t pb = (uint32_t)i & 1u;
-      if (i >= 2) ok = ok && mbar_wait(&sm.o_done[pb], (uint32_t)((i - 2) >> 1) & 1u, ctl, 0x2405);
-      const bool any_rescale = __any_sync(0xffffffffu, rescale);
-      if (any_rescale && i >= 1)
-        ok = ok && mbar_wait(&sm.o_done[pb ^ 1u], (uint32_t)((i - 1) >> 1) & 1u, ctl, 0x2406);
+      // P V of the previous tile must be done before O is rescaled and P replaced
+      if (i >= 1) ok = ok && mbar_wait(sm.o_done, (uint32_t)(i - 1) & 1u, ctl, 0x2405);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
-        if (any_rescale) {
-          tc_fence_after();
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll 1
           for (int cc = 0; cc < 4; ++cc) {
             uint32_t o[32];
@@ -396,28 +405,23 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_decode_kernel(const A
             for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
             tmem_st_32x32b_x32(tmem + (lrow << 16) + col, o);
           }
-          tmem_wait_st();
-          tc_fence_before();
         }
-        // row h of the 128-byte swizzled K-major A operand: keys 32g..32g+31
-        // are 16-byte chunks 4g..4g+3 of the row
-        uint8_t* pbase = sm.pbuf + pb * kPBytes;
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<uint4*>(pbase + swz_off(h, 4u * g + (uint32_t)j)) =
-              make_uint4(p[4 * j], p[4 * j + 1], p[4 * j + 2], p[4 * j + 3]);
-        fence_proxy_async_smem();
+        // keys 32g..32g+31 of the tile are P columns 16g..16g+15 (bf16 pairs)
+        tmem_st_32x32b_x16(tmem + (lrow << 16) + kTmemP + 16u * g, p);
+        tmem_wait_st();
+        tc_fence_before();
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full[pb]);
+      if (lane == 0) mbar_arrive(sm.p_full);
     }
+    if (leader) bulk_wait_read_all();
     // output: O / l for this warpgroup's value columns; lse from rank 0
     if (g == 1) sm.lsum[h] = l_run;
     named_bar_sync(kBarSoft, kSoftWarps * 32);
     if (g == 0) sm.lsum[h] += l_run;
     named_bar_sync(kBarSoft, kSoftWarps * 32);
     const float l_tot = sm.lsum[h];
-    if (T >= 1) ok = ok && mbar_wait(&sm.o_done[(T - 1) & 1], (uint32_t)((T - 1) >> 1) & 1u, ctl, 0x2407);
+    if (T >= 1) ok = ok && mbar_wait(sm.o_done, (uint32_t)(T - 1) & 1u, ctl, 0x2407);
     ok = __all_sync(0xffffffffu, ok);
     const float inv_l = l_tot > 0.0f ? 1.0f / l_tot : 0.0f;
     uint16_t* orow = a.out + ((int64_t)b * kHeads + h) * kDv + 256 * rank + 128 * g;
@@ -477,16 +481,14 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_decode_kernel(const A
     if (lane == 0) {
       bool ok = true;
       for (int i = 0; i < T && ok; ++i) {
-        const uint32_t pb = (uint32_t)i & 1u;
-        if (!(ok = mbar_wait(&sm.p_full[pb], (uint32_t)(i >> 1) & 1u, ctl, 0x2413))) break;
+        if (!(ok = mbar_wait(sm.p_full, (uint32_t)i & 1u, ctl, 0x2413))) break;
         tc_fence_after();
         const uint32_t sbase = smem_u32(sm.swz + (i % kSwz) * kSwzBytes);
-        const uint32_t pbase = smem_u32(sm.pbuf + pb * kPBytes);
 #pragma unroll
         for (int t = 0; t < 4; ++t)
-          mma_bf16_ss(tmem + kTmemO, smem_desc_sw128(pbase + 32u * t), smem_desc_sw128_mn(sbase + 2048u * t, kSlotBytes),
+          mma_bf16_ts(tmem + kTmemO, tmem + kTmemP + 8u * t, smem_desc_sw128_mn(sbase + 2048u * t, kSlotBytes),
                       kIdescPV, (i > 0 || t > 0) ? 1u : 0u);
-        tc_commit(&sm.o_done[pb]);
+        tc_commit(sm.o_done);
         tc_commit(&sm.swz_empty[i % kSwz]);
       }
       tc_commit(&sm.drain[1]);

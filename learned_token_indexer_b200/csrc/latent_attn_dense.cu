@@ -17,10 +17,13 @@
 // cluster of two CTAs splits the latent columns: CTA r keeps value columns
 // [256r, 256r + 256) and rope columns [512 + 32r, +32), forms partial logits
 // over them, and the two partials are exchanged through distributed shared
-// memory (st.async, double-buffered) and added, so both CTAs take identical
-// softmax decisions and each accumulates its half of O.  Key tiles of 64
-// positions arrive by TMA 2-D tile loads straight into the 128-byte swizzled
-// layout (three stages).
+// memory and added, so both CTAs take identical softmax decisions and each
+// accumulates its half of O.  The exchange is one 16 KB TMA bulk copy per
+// warpgroup and tile from a local staging buffer into the other CTA's
+// (double-buffered) receive buffer, counted by its mbarrier: per-thread
+// 16-byte remote stores moved only about 8 bytes per clock and slowed the
+// MMAs' shared-memory reads.  Key tiles of 64 positions arrive by TMA 2-D
+// tile loads straight into the 128-byte swizzled layout (two stages).
 //
 // Warps: 0-7 softmax and output (warpgroup g: keys 32g..32g+31 of a tile,
 // output columns 128g..128g+127; thread h owns row h = TMEM lane h), 8 issues
@@ -42,17 +45,18 @@ constexpr int kH = 16;
 constexpr int kTok = kRows / kH;       // 8
 constexpr int kDqk = 576, kDv = 512;
 constexpr int kTile = 64;              // keys per tile: N of the logits, K of P V
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 constexpr int kSlotBytes = kTile * 128;
 constexpr int kStageBytes = 5 * kSlotBytes;              // 4 value blocks + the rope block
 constexpr int kPBytes = kRows * kTile * 2;
-constexpr int kXPitch = 272;
-constexpr int kXBytes = kRows * kXPitch;
-constexpr uint32_t kXTx = kRows * kTile * 4;
+constexpr int kXHalf = kRows * 32 * 4;                   // one warpgroup's partial logits (16 KB)
+constexpr int kXBytes = 2 * kXHalf;
+constexpr uint32_t kXTx = kXBytes;
 constexpr int kSoftWarps = 8;
 constexpr int kMmaWarp = 8, kPvWarp = 9, kTmaWarp = 10;
 constexpr int kThreads = 11 * 32;
-constexpr uint32_t kBarSoft = 2;
+constexpr uint32_t kBarSoft = 2;                          // all softmax warps
+constexpr uint32_t kBarHalf0 = 3;                         // + g: the softmax warps of warpgroup g
 
 constexpr uint32_t kTmemO = 0;
 constexpr uint32_t kTmemQ = 256;
@@ -67,6 +71,7 @@ struct Smem {
   uint8_t* stage;      // kStages x kStageBytes, 1024-aligned
   uint8_t* pbuf;       // 2 x kPBytes
   uint8_t* x;          // 2 x kXBytes: the other CTA's partial logits of tiles i % 2
+  uint8_t* xs;         // kXBytes: this CTA's partial logits, staged for the copy
   float* tmax;         // 2 x 2 x kRows
   float* lsum;         // kRows
   uint64_t* full;      // kStages
@@ -84,7 +89,7 @@ struct Smem {
 constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 2 + 2;
 
 __host__ __device__ constexpr size_t smem_bytes() {
-  return 1024 + (size_t)kStages * kStageBytes + 2 * kPBytes + 2 * kXBytes + 5 * kRows * 4 + kNumBars * 8 + 64;
+  return 1024 + (size_t)kStages * kStageBytes + 2 * kPBytes + 3 * kXBytes + 5 * kRows * 4 + kNumBars * 8 + 64;
 }
 
 __device__ __forceinline__ Smem carve(uint8_t* raw) {
@@ -96,6 +101,8 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   p += 2 * kPBytes;
   s.x = p;
   p += 2 * kXBytes;
+  s.xs = p;
+  p += kXBytes;
   s.tmax = reinterpret_cast<float*>(p);
   p += 4 * kRows * 4;
   s.lsum = reinterpret_cast<float*>(p);
@@ -218,9 +225,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = a.q_offset + i_row;               // absolute position of the row's token
     const bool use_sel = a.sel_bits != nullptr && t + 1 > a.k;
     const uint64_t* sel = use_sel ? a.sel_bits + ((int64_t)b * a.nq + i_row) * a.kv_tiles : nullptr;
-    const uint32_t x_off = h * kXPitch + g * 128u;
-    const uint32_t x_peer0 = map_to_cta(smem_u32(sm.x + x_off), peer);
+    // row h of a warpgroup's 16 KB block of partial logits: 128 bytes, its
+    // 16-byte chunks XOR-swizzled by h so that 8 rows cover every bank
+    const uint32_t x_row = g * (uint32_t)kXHalf + h * 128u;
+    const uint32_t x_peer0 = map_to_cta(smem_u32(sm.x + g * kXHalf), peer);
     const uint32_t xfull_peer0 = map_to_cta(smem_u32(&sm.x_full[0]), peer);
+    const bool leader = (tid & 127u) == 0u;       // issues its warpgroup's copy
     const float cs = a.scale_log2;
     float m_run = -INFINITY, l_run = 0.0f;
     bool ok = true;
@@ -249,18 +259,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(sm.s_empty);
+      // stage this warpgroup's partial logits (after its previous copy has
+      // read the staging buffer), then one bulk copy into the other CTA
+      if (leader) bulk_wait_read_all();
+      named_bar_sync(kBarHalf0 + g, 128);
       if (ok) {
-        const uint32_t dst = x_peer0 + xs * kXBytes;
-        const uint32_t bar = xfull_peer0 + xs * 8u;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) st_async_v4(dst + 16 * j, s[4 * j], s[4 * j + 1], s[4 * j + 2], s[4 * j + 3], bar);
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<float4*>(sm.xs + x_row + ((j ^ (h & 7u)) << 4)) =
+              make_float4(s[4 * j], s[4 * j + 1], s[4 * j + 2], s[4 * j + 3]);
+        fence_proxy_async_smem();
+      }
+      named_bar_sync(kBarHalf0 + g, 128);
+      if (leader && ok) {
+        bulk_s2cluster(x_peer0 + xs * kXBytes, smem_u32(sm.xs + g * kXHalf), kXHalf, xfull_peer0 + xs * 8u);
+        bulk_commit_group();
       }
       ok = ok && mbar_wait_cluster(&sm.x_full[xs], (uint32_t)(i >> 1) & 1u, ctl, 0x2502);
       if (ok) {
-        const float4* xr = reinterpret_cast<const float4*>(sm.x + xs * kXBytes + x_off);
+        const uint8_t* xr = sm.x + xs * kXBytes + x_row;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float4 v = xr[j];
+          const float4 v = *reinterpret_cast<const float4*>(xr + ((j ^ (h & 7u)) << 4));
           s[4 * j] += v.x;
           s[4 * j + 1] += v.y;
           s[4 * j + 2] += v.z;
@@ -341,6 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[pb]);
     }
+    if (leader) bulk_wait_read_all();
     if (g == 1) sm.lsum[h] = l_run;
     named_bar_sync(kBarSoft, kSoftWarps * 32);
     if (g == 0) sm.lsum[h] += l_run;

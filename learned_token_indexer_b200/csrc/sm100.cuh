@@ -412,3 +412,21 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes
 }
 
 }  // namespace dsa
+
+namespace dsa {
+
+// Bulk copy of `bytes` (a multiple of 16) from this CTA's shared memory into
+// another CTA of the cluster (both addresses 16-byte aligned); the bytes
+// count against the transaction count of `remote_bar` in that CTA.
+__device__ __forceinline__ void bulk_s2cluster(uint32_t remote_dst, uint32_t local_src, uint32_t bytes,
+                                               uint32_t remote_bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(remote_dst),
+      "r"(local_src), "r"(bytes), "r"(remote_bar)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk copy of this thread has finished reading its source.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+}  // namespace dsa
