@@ -217,8 +217,12 @@ class PrefillRun:
                 ev["indexer_topk_prefill"].append((e0, e1))
                 ev[self.attn_name].append((e1, e2))
             triv = c0 < w.k
-            # indexer (+ trivial rows), attention (+ memset and selection bits on the dense path)
-            launches += 2 + (1 if triv else 0) + (2 if self.attn_name == "dense_attn" else 0)
+            # this library's kernels: the indexer when some row of the chunk has
+            # t + 1 > k, the trivial-row fill, the attention, and on the dense
+            # path the selection bits (its buffer is cleared by a memset)
+            scored = c1 > w.k
+            bits = self.attn_name == "dense_attn" and scored
+            launches += (1 if scored else 0) + (1 if triv else 0) + 1 + (1 if bits else 0)
         self.launches_per_step = launches
 
     @staticmethod
@@ -1020,6 +1024,9 @@ def main():
     ap.add_argument("--no-subs", action="store_true")
     ap.add_argument("--sub-steps", type=int, default=50)
     ap.add_argument("--sub-cpu-budget", type=float, default=10.0)
+    ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
+                    help="override a field of the main workload (e.g. B=8, L_max=8192) for a smaller case, "
+                         "such as a profiler capture")
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -1028,6 +1035,15 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.set:
+        base = W.ALL[args.workload]
+        changes = {}
+        for kv in args.set:
+            key, _, val = kv.partition("=")
+            if not hasattr(base, key):
+                ap.error(f"--set: workload has no field {key!r}")
+            changes[key] = type(getattr(base, key))(val)
+        W.ALL[args.workload] = dataclasses.replace(base, **changes)
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -364,7 +364,10 @@ dsa_status dsa_attn_dense_prefill(int B, int nq, int q_offset, int kv_len, int H
   a.kv_tiles = (kv_len + 63) / 64;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.q = static_cast<const uint16_t*>(q);
-  a.sel_bits = idx ? reinterpret_cast<const uint64_t*>(static_cast<char*>(workspace) + kHeader) : nullptr;
+  // rows with t + 1 <= k select their whole history: a chunk made only of
+  // such rows needs no selection bits
+  const bool need_bits = idx != nullptr && (int64_t)q_offset + nq > k;
+  a.sel_bits = need_bits ? reinterpret_cast<const uint64_t*>(static_cast<char*>(workspace) + kHeader) : nullptr;
   a.out = static_cast<uint16_t*>(out);
   a.lse = lse;
   a.status = status_of(workspace);

@@ -487,15 +487,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Selection bitmask of the rows that need one (t + 1 > k): bit s of word
 // [b, i, s / 64] is set when row i selected position s.  Indices outside
 // [-1, kv_len) are skipped and reported.
-__global__ void selection_bits_kernel(int B, int nq, int q_offset, int kv_len, int k, int kv_tiles,
+__global__ void selection_bits_kernel(int B, int nq, int q_offset, int kv_len, int k, int kv_tiles, int i0,
                                       const int32_t* __restrict__ idx, unsigned long long* __restrict__ bits,
                                       DeviceStatus* status) {
-  const int64_t total = (int64_t)B * nq * k;
+  // rows i0 .. nq-1 of each sequence (the first rows with t + 1 > k)
+  const int per_seq = nq - i0;
+  const int64_t total = (int64_t)B * per_seq * k;
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = e / k;
-    const int i = (int)(row % nq);
-    if (q_offset + i + 1 <= k) continue;
-    const int p = idx[e];
+    const int64_t rr = e / k;
+    const int b = (int)(rr / per_seq);
+    const int64_t row = (int64_t)b * nq + i0 + (rr - (int64_t)b * per_seq);
+    const int p = idx[row * k + (e - rr * k)];
     if (p == -1) continue;
     if (p < 0 || p >= kv_len) {
       report_status(status, kStatusDeviceCheck, 0xA77E);
@@ -537,12 +539,14 @@ size_t latent_attn_dense_smem() { return smem_bytes(); }
 cudaError_t launch_latent_attn_dense(const CUtensorMap& tmap_lat, const DenseAttnArgs& a, const int32_t* idx,
                                      cudaStream_t stream) {
   if (a.sel_bits != nullptr) {
+    // only rows with t + 1 > k read a selection: i >= k - q_offset
+    const int i0 = a.k - a.q_offset > 0 ? a.k - a.q_offset : 0;
     cudaError_t e = cudaMemsetAsync(const_cast<uint64_t*>(a.sel_bits), 0,
                                     (size_t)a.B * a.nq * a.kv_tiles * sizeof(uint64_t), stream);
     if (e != cudaSuccess) return e;
-    const int64_t total = (int64_t)a.B * a.nq * a.k;
+    const int64_t total = (int64_t)a.B * (a.nq - i0) * a.k;
     const int grid = (int)((total + 255) / 256 < 4096 ? (total + 255) / 256 : 4096);
-    selection_bits_kernel<<<grid, 256, 0, stream>>>(a.B, a.nq, a.q_offset, a.kv_len, a.k, a.kv_tiles, idx,
+    selection_bits_kernel<<<grid, 256, 0, stream>>>(a.B, a.nq, a.q_offset, a.kv_len, a.k, a.kv_tiles, i0, idx,
                                                     reinterpret_cast<unsigned long long*>(const_cast<uint64_t*>(a.sel_bits)),
                                                     a.status);
     e = cudaGetLastError();
