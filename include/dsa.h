@@ -18,7 +18,9 @@
  *    token (the dequantised value is code * scale; §2 keeps the indexer key
  *    cache quantised, with its scales).
  *  - Base pointers of the indexer operands (qI, kI) must be 16-byte aligned
- *    (they are read with TMA); other tensors need their natural alignment.
+ *    (they are read with TMA); so must w in the decode step and the score
+ *    matrix entry point (each token's head weights are staged by a bulk
+ *    copy); other tensors need their natural alignment.
  *  - Positions are 0-based.  A query at absolute position t may select keys
  *    0..t (the current token included).  Index outputs have width k: the
  *    min(k, t+1) selected positions first, in unspecified order, then -1.
@@ -102,8 +104,22 @@ dsa_status dsa_read_device_status(void* workspace, void* stream, uint32_t* detai
  * Supported: HI in {4, 8, 16, 32, 64}; dI <= 128 and a multiple of 8 (bf16)
  * or 16 (FP8); k >= 1.  Chunked prefill = several calls with increasing
  * q_offset over the same kI / workspace.
+ * Workspace.  dsa_indexer_topk_prefill_workspace() is bounded independently
+ * of the history past 16384 keys: each token streams at most 16384 candidate
+ * (score, position) pairs (SMs x 12 x 16384 x 8 B, about 0.23 GB on 148
+ * SMs), plus a second-pass area of 64 score rows.  A row whose candidates
+ * outgrow that buffer (scores with very many near-ties at its cut-off) is
+ * finished by the second pass: its score row is recomputed into the
+ * workspace, 64 rows at a time, and selected there by the row top-k (the
+ * same selection, from the same eq. (1) scores up to fp32 summation order).
+ * With kv_len > 16384 the call therefore reads the overflow count back and
+ * synchronises `stream` once.  A workspace of at least
+ * dsa_indexer_topk_prefill_workspace_full() bytes (candidate buffers sized
+ * for the whole history: no overflow, no synchronisation, the size grows
+ * with kv_len) selects that mode instead.
  * ---------------------------------------------------------------------- */
 size_t dsa_indexer_topk_prefill_workspace(int B, int nq, int kv_len, int HI, int dI, int k, int dtype);
+size_t dsa_indexer_topk_prefill_workspace_full(int B, int nq, int kv_len, int HI, int dI, int k, int dtype);
 dsa_status dsa_indexer_topk_prefill(int B, int nq, int q_offset, int kv_len, int HI, int dI, int k, int dtype,
                                     const void* qI, const float* q_scale, const void* kI, const float* k_scale,
                                     const float* w, int32_t* idx_out, float* score_out, void* workspace,

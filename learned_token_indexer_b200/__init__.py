@@ -124,12 +124,17 @@ def get_wait_timeout_ns() -> int:
 
 def indexer_topk_prefill(qI, kI, w, k: int, q_offset: int = 0, q_scale=None, k_scale=None,
                          idx_out=None, score_out=None, return_scores: bool = False,
-                         workspace: Optional[Workspace] = None):
+                         workspace: Optional[Workspace] = None, full_workspace: bool = False):
     """Fused eq. (1) + eq. (2) for a prefill chunk.
 
     qI [B, nq, HI, dI], kI [B, kv_len, dI] (bf16, or e4m3 with q_scale [B, nq]
     and k_scale [B, kv_len]), w [B, nq, HI] fp32.  Returns idx [B, nq, k]
-    int32 (and scores [B, nq, k] fp32 if asked)."""
+    int32 (and scores [B, nq, k] fp32 if asked).
+
+    The default workspace is bounded past 16384 keys (rows whose candidates
+    outgrow it take a second pass, and the call synchronises once);
+    full_workspace=True sizes the candidate buffers for the whole history
+    (no second pass, no synchronisation, memory grows with kv_len)."""
     B, nq, HI, dI = qI.shape
     kv_len = kI.shape[1]
     dt = _dtype_code(qI)
@@ -139,11 +144,14 @@ def indexer_topk_prefill(qI, kI, w, k: int, q_offset: int = 0, q_scale=None, k_s
     if return_scores and score_out is None:
         score_out = torch.empty((B, nq, k), dtype=torch.float32, device=dev)
     L = lib()
-    need = L.dsa_indexer_topk_prefill_workspace(B, nq, kv_len, HI, dI, k, dt)
+    size = L.dsa_indexer_topk_prefill_workspace_full if full_workspace else L.dsa_indexer_topk_prefill_workspace
+    need = size(B, nq, kv_len, HI, dI, k, dt)
     wsb = _ws(workspace, dev).get(need)
+    # exactly `need` bytes: the library picks the capped or the full-history
+    # mode from the size it is given
     _check(L.dsa_indexer_topk_prefill(B, nq, q_offset, kv_len, HI, dI, k, dt, _ptr(qI), _ptr(q_scale), _ptr(kI),
                                       _ptr(k_scale), _ptr(w), _ptr(idx_out), _ptr(score_out), _ptr(wsb),
-                                      wsb.numel(), _stream(dev)))
+                                      need, _stream(dev)))
     return (idx_out, score_out) if score_out is not None else idx_out
 
 

@@ -19,6 +19,7 @@ SIGNATURES = {
     "dsa_workspace_init": (_i, [_p, _sz, _p]),
     "dsa_read_device_status": (_i, [_p, _p, C.POINTER(C.c_uint32)]),
     "dsa_indexer_topk_prefill_workspace": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
+    "dsa_indexer_topk_prefill_workspace_full": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "dsa_indexer_topk_prefill": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "dsa_sparse_attn_workspace": (_sz, []),
     "dsa_sparse_attn_prefill": (_i, [_i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _p, _p, _p, _sz, _p]),

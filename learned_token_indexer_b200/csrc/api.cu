@@ -161,11 +161,36 @@ size_t dsa_small_workspace(void) { return kHeader; }
 size_t dsa_sparse_attn_workspace(void) { return kHeader; }
 
 // ---------------------------------------------------------------- prefill
-size_t dsa_indexer_topk_prefill_workspace(int B, int nq, int kv_len, int HI, int dI, int k, int dtype) {
+// Streamed candidates kept per token (4 warp sub-buffers of a quarter each);
+// rows whose candidates outgrow them are finished by the second pass, which
+// recomputes kRepairRows score rows at a time.
+static constexpr int64_t kPrefillCandCap = 16384;
+static constexpr int kScanChunkTiles = 8;   // key tiles per work item of the indexer scan
+static constexpr int kRepairRows = 64;
+
+static size_t history_cap(int kv_len) { return round_up((size_t)(kv_len > 0 ? kv_len : 1), 128); }
+
+// candidates of the 8 tokens of a block, then one cut-off scratch per epilogue group
+static size_t prefill_cand_bytes(size_t cap) {
+  return (size_t)sm_count() * (dsa::prefill_block_tokens() + 4) * cap * sizeof(uint2);
+}
+
+// The second pass: overflow count (16 B), overflow list [B * nq], then
+// kRepairRows score rows of kv_len fp32.
+static size_t prefill_repair_bytes(int B, int nq, int kv_len) {
+  return 256 + round_up((size_t)B * (size_t)(nq > 0 ? nq : 0) * 4, 256) +
+         (size_t)kRepairRows * (size_t)(kv_len > 0 ? kv_len : 1) * 4;
+}
+
+size_t dsa_indexer_topk_prefill_workspace_full(int B, int nq, int kv_len, int HI, int dI, int k, int dtype) {
   (void)B; (void)nq; (void)HI; (void)dI; (void)k; (void)dtype;
-  const size_t cap = round_up((size_t)(kv_len > 0 ? kv_len : 1), 128);   // 4 warp sub-buffers of cap / 4
-  // candidates of the 8 tokens of a block, then one cut-off scratch per epilogue group
-  return kHeader + (size_t)sm_count() * (dsa::prefill_block_tokens() + 4) * cap * sizeof(uint2);
+  return kHeader + prefill_cand_bytes(history_cap(kv_len));
+}
+
+size_t dsa_indexer_topk_prefill_workspace(int B, int nq, int kv_len, int HI, int dI, int k, int dtype) {
+  const size_t full = dsa_indexer_topk_prefill_workspace_full(B, nq, kv_len, HI, dI, k, dtype);
+  if ((int64_t)history_cap(kv_len) <= kPrefillCandCap) return full;
+  return std::min(full, kHeader + prefill_cand_bytes((size_t)kPrefillCandCap) + prefill_repair_bytes(B, nq, kv_len));
 }
 
 dsa_status dsa_indexer_topk_prefill(int B, int nq, int q_offset, int kv_len, int HI, int dI, int k, int dtype,
@@ -190,6 +215,8 @@ dsa_status dsa_indexer_topk_prefill(int B, int nq, int q_offset, int kv_len, int
   cudaStream_t s = (cudaStream_t)stream;
   const int eb = fp8 ? 1 : 2;
   const int QB = dsa::prefill_block_tokens();
+  // capped candidate buffers unless the workspace holds the full-history ones
+  const bool capped = workspace_bytes < dsa_indexer_topk_prefill_workspace_full(B, nq, kv_len, HI, dI, k, dtype);
 
   dsa::PrefillArgs a{};
   a.B = B;
@@ -212,8 +239,11 @@ dsa_status dsa_indexer_topk_prefill(int B, int nq, int q_offset, int kv_len, int
   a.idx_out = idx_out;
   a.score_out = score_out;
   a.cand = reinterpret_cast<uint2*>(static_cast<char*>(workspace) + kHeader);
-  a.cand_cap = (int64_t)round_up((size_t)kv_len, 128);
+  a.cand_cap = capped ? kPrefillCandCap : (int64_t)history_cap(kv_len);
   a.bnd = a.cand + (int64_t)sm_count() * dsa::prefill_block_tokens() * a.cand_cap;
+  char* repair = static_cast<char*>(workspace) + kHeader + prefill_cand_bytes((size_t)a.cand_cap);
+  a.ovf_count = capped ? reinterpret_cast<uint32_t*>(repair) : nullptr;
+  a.ovf_list = capped ? reinterpret_cast<int32_t*>(repair + 256) : nullptr;
   a.status = status_of(workspace);
   a.timeout_ns = g_timeout_ns;
 
@@ -229,8 +259,63 @@ dsa_status dsa_indexer_topk_prefill(int B, int nq, int q_offset, int kv_len, int
   const int kblocks = (dI * eb + 127) / 128;
   const int items = B * (a.nblk - a.first_blk);
   const int grid = std::min(sm_count(), items);
+  if (capped) {
+    cudaError_t e = cudaMemsetAsync(a.ovf_count, 0, sizeof(uint32_t), s);
+    if (e != cudaSuccess) return cuda_fail(e, "overflow count reset");
+  }
   cudaError_t e = dsa::launch_indexer_topk_prefill(HI, fp8, kblocks, tq, tk, a, grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "indexer_topk_prefill launch");
+  if (!capped) return DSA_OK;
+
+  // Second pass for the rows whose candidates outgrew their buffers: their
+  // score rows are recomputed (indexer scan over the row list) and selected
+  // with the row top-k, kRepairRows at a time.
+  uint32_t n_ovf = 0;
+  e = cudaMemcpyAsync(&n_ovf, a.ovf_count, sizeof(n_ovf), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "overflow count read-back");
+  if (n_ovf > (uint32_t)B * (uint32_t)nq) return fail(DSA_ERR_DEVICE_CHECK, "overflow count %u above %d rows", n_ovf, B * nq);
+  if (n_ovf == 0) return DSA_OK;
+  float* rscores = reinterpret_cast<float*>(repair + 256 + round_up((size_t)B * nq * 4, 256));
+  for (uint32_t r0 = 0; r0 < n_ovf; r0 += kRepairRows) {
+    const int nr = (int)std::min<uint32_t>(kRepairRows, n_ovf - r0);
+    dsa::ScanArgs sa{};
+    sa.mode = 0;
+    sa.rows = nr;
+    sa.nq = nq;
+    sa.q_offset = q_offset;
+    sa.kv_len = kv_len;
+    sa.ksteps = a.ksteps;
+    sa.chunk_tiles = kScanChunkTiles;
+    sa.max_chunks = std::max(1, ((kv_len + 127) / 128 + kScanChunkTiles - 1) / kScanChunkTiles);
+    sa.balanced = 0;
+    sa.w = w;
+    sa.q_scale = a.q_scale;
+    sa.k_scale = a.k_scale;
+    sa.out = rscores;
+    sa.row_list = a.ovf_list + r0;
+    sa.status = a.status;
+    sa.timeout_ns = g_timeout_ns;
+    CUtensorMap tq1;
+    const int box_rows = HI < 16 ? 16 : HI;
+    if (dsa_status st = make_tmap(&tq1, qI, eb, (uint64_t)dI, (uint64_t)B * nq * HI, box_rows)) return st;
+    e = dsa::launch_indexer_scan(HI, fp8, kblocks, tq1, tk, sa, std::min(sm_count(), nr * sa.max_chunks), s);
+    if (e != cudaSuccess) return cuda_fail(e, "indexer_scan (second pass) launch");
+    dsa::TopkRowsArgs t{};
+    t.rows = nr;
+    t.k = k;
+    t.scores = rscores;
+    t.row_stride = kv_len;
+    t.ncols = kv_len;
+    t.row_list = sa.row_list;
+    t.nq = nq;
+    t.q_offset = q_offset;
+    t.idx_out = idx_out;
+    t.val_out = score_out;
+    t.status = a.status;
+    e = dsa::launch_topk_rows(t, s);
+    if (e != cudaSuccess) return cuda_fail(e, "topk_rows (second pass) launch");
+  }
   return DSA_OK;
 }
 
@@ -424,7 +509,6 @@ dsa_status dsa_mass_coverage(int rows, int H, const float* lse_sparse, const flo
 }
 
 // ---------------------------------------------------------------- decode indexer
-static constexpr int kScanChunkTiles = 8;
 
 size_t dsa_indexer_topk_decode_workspace(int B, int HI, int dI, int k, int dtype, int64_t total_len, int max_len) {
   (void)B; (void)HI; (void)dI; (void)k; (void)dtype; (void)max_len;
@@ -440,7 +524,8 @@ dsa_status dsa_indexer_topk_decode(int B, int HI, int dI, int k, int dtype, cons
             "need B >= 0, k >= 1, total_len >= 0, max_len >= 0");
   DSA_CHECK(total_len < INT32_MAX && (int64_t)B * HI < INT32_MAX, DSA_ERR_UNSUPPORTED, "cache rows exceed 2^31");
   DSA_CHECK(qI && w && kI_cache && cu_seqlens && idx_out, DSA_ERR_INVALID_ARG, "null tensor pointer");
-  DSA_CHECK(aligned(qI, 16) && aligned(kI_cache, 16), DSA_ERR_INVALID_ARG, "qI and kI_cache must be 16-byte aligned");
+  DSA_CHECK(aligned(qI, 16) && aligned(kI_cache, 16) && aligned(w, 16), DSA_ERR_INVALID_ARG,
+            "qI, kI_cache and w must be 16-byte aligned");
   const bool fp8 = dtype == DSA_FP8_E4M3;
   DSA_CHECK(!fp8 || (q_scale && k_scale), DSA_ERR_INVALID_ARG, "FP8 needs q_scale and k_scale");
   const size_t need = dsa_indexer_topk_decode_workspace(B, HI, dI, k, dtype, total_len, max_len);
@@ -499,7 +584,8 @@ dsa_status dsa_indexer_scores(int B, int nq, int q_offset, int kv_len, int HI, i
   DSA_CHECK((int64_t)B * nq * HI < INT32_MAX && (int64_t)B * kv_len < INT32_MAX, DSA_ERR_UNSUPPORTED,
             "tensor rows exceed 2^31");
   DSA_CHECK(qI && kI && w && scores, DSA_ERR_INVALID_ARG, "null tensor pointer");
-  DSA_CHECK(aligned(qI, 16) && aligned(kI, 16), DSA_ERR_INVALID_ARG, "qI and kI must be 16-byte aligned");
+  DSA_CHECK(aligned(qI, 16) && aligned(kI, 16) && aligned(w, 16), DSA_ERR_INVALID_ARG,
+            "qI, kI and w must be 16-byte aligned");
   const bool fp8 = dtype == DSA_FP8_E4M3;
   DSA_CHECK(!fp8 || (q_scale && k_scale), DSA_ERR_INVALID_ARG, "FP8 needs q_scale and k_scale");
   if (dsa_status st = check_ws(workspace, workspace_bytes, kHeader)) return st;

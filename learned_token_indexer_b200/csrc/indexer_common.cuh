@@ -98,12 +98,16 @@ __device__ __forceinline__ void group_head_sums(uint32_t taddr, const float* w_s
   for (int u = 0; u < NU; ++u) {
     if (u + 1 < NU) load(u + 1, buf[(u + 1) & 1]);
     const int j = u / UPT;
-    const float2* w = reinterpret_cast<const float2*>(w_smem + j * HI + (u % UPT) * UW);
+    const float4* w = reinterpret_cast<const float4*>(w_smem + j * HI + (u % UPT) * UW);
 #pragma unroll
-    for (int h = 0; h < UW; h += 2) {
-      const float2 x = make_float2(fmaxf(__uint_as_float(buf[u & 1][h]), 0.0f),
-                                   fmaxf(__uint_as_float(buf[u & 1][h + 1]), 0.0f));
-      part[j][(h >> 1) & 1] = ffma2(w[h >> 1], x, part[j][(h >> 1) & 1]);
+    for (int h = 0; h < UW; h += 4) {
+      const float4 w4 = w[h >> 2];   // four heads' weights in one shared load
+      const float2 x0 = make_float2(fmaxf(__uint_as_float(buf[u & 1][h]), 0.0f),
+                                    fmaxf(__uint_as_float(buf[u & 1][h + 1]), 0.0f));
+      const float2 x1 = make_float2(fmaxf(__uint_as_float(buf[u & 1][h + 2]), 0.0f),
+                                    fmaxf(__uint_as_float(buf[u & 1][h + 3]), 0.0f));
+      part[j][0] = ffma2(make_float2(w4.x, w4.y), x0, part[j][0]);
+      part[j][1] = ffma2(make_float2(w4.z, w4.w), x1, part[j][1]);
     }
     if (u + 1 < NU) {
       tmem_wait_ld(buf[(u + 1) & 1]);

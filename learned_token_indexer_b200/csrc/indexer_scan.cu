@@ -7,11 +7,13 @@
 // materialises the causal prefill score matrix for small n.
 //
 // Per CTA: warp 0 = TMA producer, warp 1 = tcgen05 MMA issuer (and TMEM
-// owner), warps 2..5 = epilogue (TMEM -> ReLU * w -> head sum -> global).
-// The MMA computes D[128 keys x N] with keys on TMEM lanes and the token's
-// heads on columns; two accumulators alternate so the epilogue of one tile
-// overlaps the MMA of the next.  Work items are (row, run of key tiles),
-// spread over a persistent grid.
+// owner), warps 2..9 = two epilogue warpgroups (TMEM -> ReLU * w -> head sum
+// -> global).  The MMA computes D[128 keys x N] with keys on TMEM lanes and
+// the token's heads on columns into four accumulators used in turn; the two
+// warpgroups take alternate tiles, so two tiles' epilogues run at once while
+// the MMA fills the next ones.  Work items are (row, run of key tiles),
+// spread over a persistent grid; the producer stages each item's q^I tile and
+// its head weights w[t, :] together.
 #include "indexer_common.cuh"
 #include "kernels.h"
 
@@ -24,26 +26,32 @@ namespace {
 // 256-byte one to keep the same bytes on the way from HBM).
 template <int KB>
 constexpr int scan_stages() { return KB == 1 ? 8 : 4; }
-constexpr int kScanThreads = 192;
+constexpr int kScanThreads = 320;
 constexpr int kEpiWarp0 = 2;
+constexpr int kEpiWarps = 8;     // two warpgroups
+constexpr int kScanAcc = 4;      // accumulators in TMEM
 
 struct ScanRow {
   int64_t key_base;
   int len;
+  int qrow;      // row of q^I / w / q_scale
   float* out;
 };
 
 __device__ __forceinline__ ScanRow scan_row(const ScanArgs& a, int r) {
   ScanRow g;
   if (a.mode == 0) {
-    const int b = r / a.nq, i = r - b * a.nq;
+    const int q = a.row_list ? a.row_list[r] : r;
+    const int b = q / a.nq, i = q - b * a.nq;
     g.key_base = (int64_t)b * a.kv_len;
     g.len = a.q_offset + i + 1;
+    g.qrow = q;
     g.out = a.out + (int64_t)r * a.kv_len;
   } else {
     const int64_t lo = a.cu_seqlens[r];
     g.key_base = lo;
     g.len = (int)(a.cu_seqlens[r + 1] - lo);
+    g.qrow = r;
     g.out = a.out + lo;
   }
   return g;
@@ -105,7 +113,10 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   constexpr int N = HI < 16 ? 16 : HI;
   constexpr int kQBytes = N * KB * kSwizzleBytes;
   constexpr int kKBytes = kTileKeys * KB * kSwizzleBytes;
-  constexpr uint32_t kTmemCols = (2 * N <= 32) ? 32 : (2 * N <= 64 ? 64 : (2 * N <= 128 ? 128 : 256));
+  constexpr uint32_t kTmemCols =
+      (kScanAcc * N <= 32) ? 32 : (kScanAcc * N <= 64 ? 64 : (kScanAcc * N <= 128 ? 128 : 256));
+  static_assert(kScanAcc * N <= 256, "accumulators exceed the TMEM allocation");
+  constexpr uint32_t kWBytes = HI * 4;
   constexpr uint32_t kIdesc = instr_desc(ElemTraits<FP8>::kFormat, kTileKeys, N);
   constexpr int kElemsPerBlock = ElemTraits<FP8>::kElemsPerBlock;
   constexpr int kScanStages = scan_stages<KB>();
@@ -114,15 +125,15 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = base;
   uint8_t* sQ = sK + kScanStages * kKBytes;
-  float* sW = reinterpret_cast<float*>(sQ + 2 * kQBytes);
+  float* sW = reinterpret_cast<float*>(sQ + 2 * kQBytes);   // [2][HI], beside the two q^I slots
   uint64_t* bars = reinterpret_cast<uint64_t*>(sW + 2 * HI);
   uint64_t* k_full = bars;
   uint64_t* k_empty = bars + kScanStages;
   uint64_t* q_full = bars + 2 * kScanStages;
   uint64_t* q_empty = q_full + 2;
   uint64_t* acc_full = q_empty + 2;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* mma_done = acc_empty + 2;
+  uint64_t* acc_empty = acc_full + kScanAcc;
+  uint64_t* mma_done = acc_empty + kScanAcc;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   int* sPre = reinterpret_cast<int*>(tmem_slot + 4);   // [rows + 1] in balanced mode
@@ -135,9 +146,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1);
+      mbar_init(&q_empty[s], 1 + kEpiWarps);   // the MMA's commit and every epilogue warp
+    }
+    for (int s = 0; s < kScanAcc; ++s) {
       mbar_init(&acc_full[s], 1);
-      mbar_init(&acc_empty[s], 4);
+      mbar_init(&acc_empty[s], 4);              // the four warps of the warpgroup that reads it
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0u;
@@ -200,10 +213,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         scan_item(a, item, row, t0, nt, g, sPre, balanced);
         if (nt == 0) continue;
         if (!(ok = mbar_wait(&q_empty[qslot], qphase ^ 1u, ctl, 0x101))) break;
-        mbar_arrive_expect_tx(&q_full[qslot], kQBytes);
+        mbar_arrive_expect_tx(&q_full[qslot], kQBytes + kWBytes);
         for (int kb = 0; kb < KB; ++kb)
           tma_load_2d(sQ + qslot * kQBytes + kb * N * kSwizzleBytes, &tmap_q, &q_full[qslot], kb * kElemsPerBlock,
-                      row * HI);
+                      g.qrow * HI);
+        bulk_copy_g2s(smem_u32(sW + qslot * HI), a.w + (int64_t)g.qrow * HI, kWBytes, &q_full[qslot]);
         q_issued[qslot] = true;
         q_last_parity[qslot] = qphase;
         if (++qslot == 2) { qslot = 0; qphase ^= 1u; }
@@ -241,8 +255,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int stage = 0, qslot = 0, acc = 0;
-      uint32_t kphase = 0, qphase = 0, aphase = 0;
+      int stage = 0, qslot = 0;
+      uint32_t kphase = 0, qphase = 0, n = 0;   // n: tile sequence number
       bool ok = true;
       for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
         int row, t0, nt;
@@ -253,6 +267,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         tc_fence_after();
         const uint32_t qaddr = smem_u32(sQ + qslot * kQBytes);
         for (int t = 0; t < nt; ++t) {
+          const uint32_t acc = n % kScanAcc, aphase = (n / kScanAcc) & 1u;
           if (!(ok = mbar_wait(&k_full[stage], kphase, ctl, 0x202))) break;
           if (!(ok = mbar_wait(&acc_empty[acc], aphase ^ 1u, ctl, 0x203))) break;
           tc_fence_after();
@@ -260,7 +275,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           tc_commit(&acc_full[acc]);
           tc_commit(&k_empty[stage]);
           if (++stage == kScanStages) { stage = 0; kphase ^= 1u; }
-          if (++acc == 2) { acc = 0; aphase ^= 1u; }
+          ++n;
         }
         if (!ok) break;
         tc_commit(&q_empty[qslot]);
@@ -276,30 +291,30 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     // Same barrier sequence for every thread; a failed wait only disables work.
-    const uint32_t ew = warp - kEpiWarp0;             // 0..3
+    // Warpgroup g takes the tiles whose sequence number n has n % 2 == g.
+    const uint32_t g = (warp - kEpiWarp0) >> 2;       // 0..1
     const uint32_t lane_grp = (warp & 3u) * 32u;      // TMEM lanes this warp may access
-    const uint32_t et = ew * 32u + lane;              // 0..127
-    int acc = 0;
-    uint32_t aphase = 0;
+    int qslot = 0;
+    uint32_t qphase = 0, n = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
       int row, t0, nt;
-      ScanRow g;
-      scan_item(a, item, row, t0, nt, g, sPre, balanced);
+      ScanRow gr;
+      scan_item(a, item, row, t0, nt, gr, sPre, balanced);
       if (nt == 0) continue;
-      named_bar_sync(1, 128);
-      if (et < (uint32_t)HI) {
-        float wv = a.w[(int64_t)row * HI + et];
-        if (FP8) wv *= a.q_scale[row];
-        sW[et] = wv;
-      }
-      named_bar_sync(1, 128);
-      for (int t = 0; t < nt; ++t) {
+      // q_scale is requested before the wait so its latency hides behind it
+      const float qs = FP8 ? __ldg(a.q_scale + gr.qrow) : 1.0f;
+      const bool gotq = ok && mbar_wait(&q_full[qslot], qphase, ctl, 0x300);
+      ok = __all_sync(0xffffffffu, gotq);
+      const float* w_row = sW + qslot * HI;
+      for (int t = 0; t < nt; ++t, ++n) {
+        if ((n & 1u) != g) continue;
+        const uint32_t acc = n % kScanAcc, aphase = (n / kScanAcc) & 1u;
         const int s = (t0 + t) * kTileKeys + (int)lane_grp + (int)lane;
         // the key's FP8 scale is requested before the wait, so its latency
         // hides behind the MMA instead of following the head sum
         float kscale = 1.0f;
-        if (FP8 && s < g.len) kscale = __ldg(a.k_scale + g.key_base + s);
+        if (FP8 && s < gr.len) kscale = __ldg(a.k_scale + gr.key_base + s) * qs;
         const bool got = ok && mbar_wait(&acc_full[acc], aphase, ctl, 0x301);
         ok = __all_sync(0xffffffffu, got);
         if (ok) {
@@ -310,14 +325,17 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[acc]);
-          if (s < g.len) {
-            float score = scan_head_sum<HI>(r, sW);
+          if (s < gr.len) {
+            float score = scan_head_sum<HI>(r, w_row);
             if (FP8) score *= kscale;
-            g.out[s] = score + 0.0f;
+            gr.out[s] = score + 0.0f;
           }
         }
-        if (++acc == 2) { acc = 0; aphase ^= 1u; }
       }
+      // this warp is done with the item's weights
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&q_empty[qslot]);
+      if (++qslot == 2) { qslot = 0; qphase ^= 1u; }
     }
   }
   tc_fence_before();
@@ -332,7 +350,7 @@ template <int HI, bool FP8, int KB>
 static size_t scan_smem_bytes() {
   constexpr int N = HI < 16 ? 16 : HI;
   return 1024 + scan_stages<KB>() * kTileKeys * KB * kSwizzleBytes + 2 * N * KB * kSwizzleBytes + 2 * HI * 4 +
-         (2 * scan_stages<KB>() + 9) * 8 + 16 + (kScanMaxBalancedRows + 1) * 4;
+         (2 * scan_stages<KB>() + 4 + 2 * kScanAcc + 1) * 8 + 16 + (kScanMaxBalancedRows + 1) * 4;
 }
 
 template <int HI, bool FP8, int KB>

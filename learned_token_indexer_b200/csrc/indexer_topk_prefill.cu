@@ -334,7 +334,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       // accepted (key, position) pairs: this warp's sub-buffer of each token
       // (warp q of the group sees keys with s mod 128 in [32q, 32q + 32))
       uint2* cand_w[2];
-      uint32_t cnt[2] = {0u, 0u};
+      uint32_t cnt[2] = {0u, 0u};   // accepted entries (stored while below sub_cap)
+      const uint32_t sub_cap = (uint32_t)(a.cand_cap / 4);
 #pragma unroll
       for (int u = 0; u < 2; ++u)
         cand_w[u] = a.cand + ((int64_t)blockIdx.x * kQB + ST(u)) * a.cand_cap + quarter * (a.cand_cap / 4);
@@ -381,7 +382,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           const bool acc = tok_valid[u] && s <= tok_t[u] && key >= floor_key;
           const uint32_t mask = __ballot_sync(0xffffffffu, acc);
           if (acc) {
-            cand_w[u][cnt[u] + __popc(mask & ((1u << lane) - 1u))] = make_uint2(key, (uint32_t)s);
+            const uint32_t slot = cnt[u] + __popc(mask & ((1u << lane) - 1u));
+            if (slot < sub_cap) cand_w[u][slot] = make_uint2(key, (uint32_t)s);
             // histogram of accepted scores, one atomic per distinct bin of the warp
             const uint32_t bin = score_bin(key);
             const uint32_t peers = __match_any_sync(mask, bin);
@@ -411,6 +413,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const int st = ST(g);
         const int kk = min(a.k, tok_t[g] + 1);
         const uint32_t c0 = sCnt[st * 4], c1 = sCnt[st * 4 + 1], c2 = sCnt[st * 4 + 2], c3 = sCnt[st * 4 + 3];
+        const int64_t row = (int64_t)blk.b * a.nq + blk.t0 + st;
+        const uint32_t sub_cap = (uint32_t)(a.cand_cap / 4);
+        if (max(max(c0, c1), max(c2, c3)) > sub_cap) {
+          // a sub-buffer overflowed (warpgroup-uniform): the row goes to the second pass
+          if (tid == 0 && a.ovf_list) a.ovf_list[atomicAdd(a.ovf_count, 1u)] = (int32_t)row;
+          continue;
+        }
         const int m = (int)(c0 + c1 + c2 + c3);
         uint32_t* hist = sHist + st * kHistBins;
         const uint2* buf = a.cand + ((int64_t)blockIdx.x * kQB + st) * a.cand_cap;
@@ -445,7 +454,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // One pass over the candidates: entries above the cut-off bin are
         // selected outright and written now; the cut-off bin's entries are
         // gathered into this group's scratch, where the refinement runs.
-        const int64_t row = (int64_t)blk.b * a.nq + blk.t0 + st;
         int32_t* idx_row = a.idx_out + row * a.k;
         float* score_row = a.score_out ? a.score_out + row * a.k : nullptr;
         uint2* bnd = a.bnd + ((int64_t)blockIdx.x * 4 + wg) * a.cand_cap;

@@ -47,6 +47,7 @@ struct ScanArgs {
   const float* q_scale;        // [rows] (FP8) or null
   const float* k_scale;        // [key rows] (FP8) or null
   float* out;                  // prefill [rows, kv_len]; decode [sum L]
+  const int32_t* row_list;     // prefill only, or null: scan row r is query row row_list[r] (b * nq + i)
   DeviceStatus* status;
   uint64_t timeout_ns;
 };
@@ -65,6 +66,11 @@ struct PrefillArgs {
   uint2* cand;                 // [grid * 8, cand_cap] candidate (key, pos) buffers
   int64_t cand_cap;
   uint2* bnd;                  // [grid * 4, cand_cap] cut-off bin entries of the row being selected
+  // Candidate overflow (cand_cap below the history): a row whose accepted
+  // entries outgrow its buffer is not selected here; its index b * nq + i is
+  // appended to ovf_list (count in *ovf_count) for a second pass.
+  uint32_t* ovf_count;
+  int32_t* ovf_list;
   DeviceStatus* status;
   uint64_t timeout_ns;
 };
@@ -79,6 +85,11 @@ struct TopkRowsArgs {
   const int64_t* cu_seqlens;   // ragged rows: row r = scores[cu[r] .. cu[r+1])
   int32_t* idx_out;            // [rows, k]
   float* val_out;              // [rows, k] or null
+  // Prefill rows given by list (row_stride layout): score row r belongs to
+  // query row q = row_list[r] = b * nq + i, has length q_offset + i + 1 and
+  // writes idx_out / val_out row q.
+  const int32_t* row_list;
+  int nq, q_offset;
   DeviceStatus* status;
 };
 

@@ -162,11 +162,6 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   return s;
 }
 
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
 
 using lattn::pack_bf16x2;
 using lattn::regs_dec;
@@ -517,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1) latent_attn_decode_kernel(const A
         const int j = i * kTile + n;
         const int p = j < a.k ? idx[j] : -1;
         const int64_t row = base + ((p >= 0 && p < L) ? p : 0);
-        bulk_g2s(dst0 + n * kRowBytes, a.latent + row * kDqk + 256 * rank, kRowBytes, &sm.raw_full[r]);
+        bulk_copy_g2s(dst0 + n * kRowBytes, a.latent + row * kDqk + 256 * rank, kRowBytes, &sm.raw_full[r]);
       }
       issued = i + 1;
     }

@@ -3,13 +3,21 @@
 // separate radix top-k that handles variable-length rows via seq_lens), plus
 // small helper kernels.
 //
-// One CTA (1024 threads) per row, two passes over the row in the usual case:
-// a histogram of the row's scores over the coarse score bins finds the
-// cut-off bin; one pass then writes every entry above that bin and gathers
-// the cut-off bin's entries into shared memory, where the exact radix
-// refinement on (key, position) runs.  (A cut-off bin too large for shared
-// memory is refined over the row instead.)  Used by the decode step (64 rows
-// of 4096..65536 scores) and by the debug path.
+// One CTA (1024 threads) per row.  A long row (at least 8192 entries and 4k)
+// first takes a 1/16 sample of itself and finds a cut-off key tau a little
+// below the sample's estimate of the k-th largest key; one 16-byte-load pass
+// over the row then gathers every entry with key >= tau into shared memory,
+// where the exact radix select of select.cuh runs.  When at least k entries
+// reach tau, every selected entry and every tie at the k-th key is among the
+// gathered ones, so the result is the row's exact top-k; when fewer than k
+// reach tau, or more than the shared buffer holds, the row falls back to the
+// two-pass path.  The two-pass path (also used for short rows): a histogram of
+// the row's scores over the coarse score bins finds the cut-off bin; one pass
+// then writes every entry above that bin and gathers the cut-off bin's
+// entries into shared memory, where the exact radix refinement on
+// (key, position) runs.  (A cut-off bin too large for shared memory is refined
+// over the row instead.)  Used by the decode step (64 rows of 4096..65536
+// scores) and by the debug path.
 #include "kernels.h"
 #include "select.cuh"
 
@@ -18,13 +26,22 @@ namespace dsa {
 namespace {
 constexpr int kRowThreads = 1024;
 constexpr int kRowBins = 2048;        // refinement digit bins
-constexpr int kBndCap = 4096;         // cut-off bin entries kept in shared memory
+constexpr int kBndCap = 4096;         // cut-off bin entries kept in shared memory (two-pass path)
+constexpr int kCandCap = 16384;       // gathered candidates (prefilter path)
+constexpr int kSampleMax = 8192;      // sampled entries
+constexpr int kGatherBatch = 4;       // 16-byte loads in flight per thread in the gather pass
+constexpr int kPrefilterMinLen = 8192;
+constexpr size_t kTopkDynSmem = (size_t)kCandCap * sizeof(uint2);
+static_assert(kBndCap <= kCandCap && kSampleMax * sizeof(uint32_t) <= kTopkDynSmem, "aliased buffers");
 }  // namespace
 
 __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRowsArgs a) {
   __shared__ uint32_t hist[kRowBins];
-  __shared__ uint2 bnd[kBndCap];
   __shared__ SelectShared<kRowThreads> sh;
+  extern __shared__ __align__(16) uint8_t topk_dyn[];
+  uint2* cand = reinterpret_cast<uint2*>(topk_dyn);     // prefilter candidates
+  uint32_t* samp = reinterpret_cast<uint32_t*>(topk_dyn);  // sample keys (before the gather)
+  uint2* bnd = cand;                                    // two-pass cut-off bin entries
   const int row = blockIdx.x;
   const uint32_t tid = threadIdx.x, lane = tid & 31u;
   const float* src;
@@ -36,6 +53,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRow
   } else {
     src = a.scores + (int64_t)row * a.row_stride;
     len = a.row_len ? a.row_len[row] : a.ncols;
+    if (a.row_list) len = a.q_offset + a.row_list[row] % a.nq + 1;
     if (len > a.ncols) {   // a row cannot be longer than the matrix
       if (threadIdx.x == 0) report_status(a.status, kStatusDeviceCheck, 0x70E1u);
       len = a.ncols;
@@ -43,8 +61,9 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRow
   }
   if (len < 0) len = 0;
   const int kk = len < a.k ? len : a.k;
-  int32_t* idx_row = a.idx_out + (int64_t)row * a.k;
-  float* val_row = a.val_out ? a.val_out + (int64_t)row * a.k : nullptr;
+  const int64_t out_row = a.row_list ? (int64_t)a.row_list[row] : (int64_t)row;
+  int32_t* idx_row = a.idx_out + out_row * a.k;
+  float* val_row = a.val_out ? a.val_out + out_row * a.k : nullptr;
   auto get = [src](int i, uint32_t& key, uint32_t& pos) {
     key = float_to_key(src[i]);
     pos = (uint32_t)i;
@@ -58,6 +77,105 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRow
     r.pos_hi = 0;
     group_emit<kRowThreads>(get, kk > 0 ? len : 0, r, kk, a.k, idx_row, val_row, sh, tid, 0, a.status);
     return;
+  }
+  // ---- prefilter for long rows
+  const int head = min(len, (int)((((16u - ((uint32_t)reinterpret_cast<uintptr_t>(src) & 15u)) & 15u)) >> 2));
+  const int nb4 = (len - head) >> 2;                    // 16-byte aligned body, in float4
+  if (len >= kPrefilterMinLen && len >= 4 * kk) {
+    const float4* body = reinterpret_cast<const float4*>(src + head);
+    const int ns4 = min(nb4 >> 4, kSampleMax / 4);
+    const int st = nb4 / ns4;                            // >= 16
+    const int s_n = 4 * ns4;
+    for (int j = (int)tid; j < ns4; j += kRowThreads) {
+      const float4 v = body[(int64_t)j * st];
+      samp[4 * j + 0] = float_to_key(v.x);
+      samp[4 * j + 1] = float_to_key(v.y);
+      samp[4 * j + 2] = float_to_key(v.z);
+      samp[4 * j + 3] = float_to_key(v.w);
+    }
+    __syncthreads();
+    // m-th largest sampled key, m about 1.25 kk s/len plus a margin, so that
+    // more than kk row entries reach it unless the sample is unrepresentative
+    const int m = (int)((5LL * kk * s_n + 4LL * len - 1) / (4LL * len)) + 32;
+    auto get_s = [samp](int i, uint32_t& key, uint32_t& pos) {
+      key = samp[i];
+      pos = (uint32_t)i;
+    };
+    const SelectResult rs = group_refine<kRowThreads, kRowBins>(get_s, s_n, 0u, 0xFFFFFFFFu, (uint32_t)m,
+                                                                (uint32_t)(s_n - 1), hist, sh, tid, 0, a.status);
+    const uint32_t tau = rs.lo;
+    if (tid == 0) sh.bnd_count = 0u;
+    __syncthreads();   // sample reads done before the buffer is reused
+    for (int j0 = 0; j0 < nb4; j0 += kRowThreads * kGatherBatch) {
+      float4 v[kGatherBatch];
+#pragma unroll
+      for (int u = 0; u < kGatherBatch; ++u) {
+        const int j = j0 + u * kRowThreads + (int)tid;
+        v[u] = j < nb4 ? body[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      uint32_t n = 0;
+#pragma unroll
+      for (int u = 0; u < kGatherBatch; ++u) {
+        const int j = j0 + u * kRowThreads + (int)tid;
+        if (j < nb4)
+          n += (float_to_key(v[u].x) >= tau) + (float_to_key(v[u].y) >= tau) + (float_to_key(v[u].z) >= tau) +
+               (float_to_key(v[u].w) >= tau);
+      }
+      uint32_t incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= (uint32_t)o) incl += t;
+      }
+      uint32_t base = 0;
+      if (lane == 31 && incl) base = atomicAdd(&sh.bnd_count, incl);
+      base = __shfl_sync(0xffffffffu, base, 31) + incl - n;
+      if (n) {
+#pragma unroll
+        for (int u = 0; u < kGatherBatch; ++u) {
+          const int j = j0 + u * kRowThreads + (int)tid;
+          const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t key = float_to_key(f[c]);
+            if (j < nb4 && key >= tau) {
+              if (base < (uint32_t)kCandCap) cand[base] = make_uint2(key, (uint32_t)(head + 4 * j + c));
+              ++base;
+            }
+          }
+        }
+      }
+    }
+    if (tid < 32) {   // the unaligned head and tail (at most 3 entries each)
+      const int tail0 = head + 4 * nb4;
+      const int i = tid < 3 ? (int)tid : tail0 + (int)tid - 3;
+      const bool valid = tid < 3 ? i < head : (tid < 6 && i < len);
+      const uint32_t key = valid ? float_to_key(src[i]) : 0u;
+      const bool take = valid && key >= tau;
+      const uint32_t mk = __ballot_sync(0xffffffffu, take);
+      uint32_t base = 0;
+      if (lane == 0 && mk) base = atomicAdd(&sh.bnd_count, (uint32_t)__popc(mk));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (take) {
+        const uint32_t slot = base + __popc(mk & ((1u << lane) - 1u));
+        if (slot < (uint32_t)kCandCap) cand[slot] = make_uint2(key, (uint32_t)i);
+      }
+    }
+    __syncthreads();
+    const uint32_t c = sh.bnd_count;
+    __syncthreads();   // every thread has read the count before the select reuses sh
+    if (c >= (uint32_t)kk && c <= (uint32_t)kCandCap) {
+      auto get_c = [cand](int i, uint32_t& key, uint32_t& pos) {
+        const uint2 e = cand[i];
+        key = e.x;
+        pos = e.y;
+      };
+      const SelectResult r = group_refine<kRowThreads, kRowBins>(get_c, (int)c, tau, 0xFFFFFFFFu, (uint32_t)kk,
+                                                                 (uint32_t)(len - 1), hist, sh, tid, 0, a.status);
+      group_emit<kRowThreads>(get_c, (int)c, r, kk, a.k, idx_row, val_row, sh, tid, 0, a.status);
+      return;
+    }
+    // the sample misjudged the row: take the two-pass path below
   }
   // ---- pass 1: coarse score-bin histogram of the row
   for (int i = (int)tid; i < kScoreBins; i += kRowThreads) hist[i] = 0u;
@@ -130,7 +248,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRow
   r.key_all_in = 1;
   r.pos_hi = 0;
   if (nb <= (uint32_t)kBndCap) {
-    auto get_bnd = [](int i, uint32_t& key, uint32_t& pos) {
+    auto get_bnd = [bnd](int i, uint32_t& key, uint32_t& pos) {
       const uint2 e = bnd[i];
       key = e.x;
       pos = e.y;
@@ -152,29 +270,44 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRow
 
 cudaError_t launch_topk_rows(const TopkRowsArgs& a, cudaStream_t stream) {
   if (a.rows == 0) return cudaSuccess;
-  topk_rows_kernel<<<a.rows, kRowThreads, 0, stream>>>(a);
+  cudaError_t e = setup_once_per_device([] {
+    return cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTopkDynSmem);
+  });
+  if (e != cudaSuccess) return e;
+  topk_rows_kernel<<<a.rows, kRowThreads, kTopkDynSmem, stream>>>(a);
   return cudaGetLastError();
 }
 
 // Rows whose history fits in the budget (t + 1 <= k) select every position:
 // S_t = {0, ..., t}, the rest of the row is -1 (eq. (2), short history).
-__global__ void fill_trivial_rows_kernel(int nq, int q_offset, int rows_per_seq, int k, int32_t* idx) {
-  const int b = blockIdx.y;
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < (int64_t)rows_per_seq * k;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int i = (int)(e / k), slot = (int)(e - (int64_t)i * k);
+// Rows whose history holds at most k positions (t + 1 <= k) select all of
+// it (eq. (2)): slot j holds j for j <= t, then -1.  One block per row (grid
+// stride), 16-byte stores when the rows are 16-byte aligned.
+__global__ void fill_trivial_rows_kernel(int nq, int q_offset, int rows_per_seq, int64_t nrows, int k, int32_t* idx,
+                                         int vec4) {
+  for (int64_t r = blockIdx.x; r < nrows; r += gridDim.x) {
+    const int b = (int)(r / rows_per_seq), i = (int)(r - (int64_t)b * rows_per_seq);
     const int t = q_offset + i;
-    idx[((int64_t)b * nq + i) * k + slot] = slot <= t ? slot : -1;
+    int32_t* row = idx + ((int64_t)b * nq + i) * k;
+    if (vec4) {
+      for (int q = threadIdx.x; q < k / 4; q += blockDim.x) {
+        const int s = 4 * q;
+        reinterpret_cast<int4*>(row)[q] =
+            make_int4(s <= t ? s : -1, s + 1 <= t ? s + 1 : -1, s + 2 <= t ? s + 2 : -1, s + 3 <= t ? s + 3 : -1);
+      }
+    } else {
+      for (int s = threadIdx.x; s < k; s += blockDim.x) row[s] = s <= t ? s : -1;
+    }
   }
 }
 
 cudaError_t launch_fill_trivial_rows(int B, int nq, int q_offset, int rows_per_seq, int k, int32_t* idx,
                                      cudaStream_t stream) {
   if (rows_per_seq <= 0 || B <= 0) return cudaSuccess;
-  const int64_t n = (int64_t)rows_per_seq * k;
-  int gx = (int)((n + 255) / 256);
-  if (gx > 4096) gx = 4096;
-  fill_trivial_rows_kernel<<<dim3(gx, B), 256, 0, stream>>>(nq, q_offset, rows_per_seq, k, idx);
+  const int64_t nrows = (int64_t)B * rows_per_seq;
+  const int vec4 = (k % 4 == 0 && (reinterpret_cast<uintptr_t>(idx) & 15u) == 0) ? 1 : 0;
+  const int grid = (int)(nrows < 148 * 8 ? nrows : 148 * 8);
+  fill_trivial_rows_kernel<<<grid, 256, 0, stream>>>(nq, q_offset, rows_per_seq, nrows, k, idx, vec4);
   return cudaGetLastError();
 }
 

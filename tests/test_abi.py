@@ -106,6 +106,22 @@ def test_workspace_sizes(lib):
     assert small == 256
     pf = lib.dsa_indexer_topk_prefill_workspace(1, 8192, 8192, 64, 128, 2048, 0)
     assert pf > 256 and (pf - 256) % (8 * 8192 * 8) == 0
+    assert pf == lib.dsa_indexer_topk_prefill_workspace_full(1, 8192, 8192, 64, 128, 2048, 0)
+
+
+def test_prefill_workspace_is_bounded_past_16384_keys(lib):
+    """Candidate buffers stop growing at 16384 entries per token; only the
+    second pass's 64 score rows (and the B * nq overflow list) follow kv_len."""
+    ws = lambda nq, kv: lib.dsa_indexer_topk_prefill_workspace(1, nq, kv, 64, 128, 2048, 0)
+    full = lambda nq, kv: lib.dsa_indexer_topk_prefill_workspace_full(1, nq, kv, 64, 128, 2048, 0)
+    sms = (full(8, 16384) - 256) // (12 * 16384 * 8)
+    assert full(8, 16384) == 256 + sms * 12 * 16384 * 8 == ws(8, 16384)
+    cand = 256 + sms * 12 * 16384 * 8
+    assert ws(8192, 131072) == cand + 256 + 8192 * 4 + 64 * 131072 * 4
+    assert ws(8192, 262144) - ws(8192, 131072) == 64 * 131072 * 4
+    assert full(8192, 131072) == 256 + sms * 12 * 131072 * 8
+    if sms == 148:
+        assert ws(8192, 131072) < 0.3e9 < 1.8e9 < full(8192, 131072)
     dec = lib.dsa_indexer_topk_decode_workspace(64, 64, 128, 2048, 0, 1000, 100)
     assert dec >= 256 + 4000
 

@@ -121,6 +121,58 @@ def test_topk_rows_exact_with_ties(k):
         assert np.array_equal(val[r, :m], s[r, idx[r, :m]].numpy() + 0.0)
 
 
+def _topk_rows_check(s, lens, k):
+    ws = _ws()
+    idx, val = dsa.topk_rows(s.cuda(), k, row_len=lens.cuda(), return_values=True, workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    idx, val = idx.cpu().numpy(), val.cpu().numpy()
+    for r in range(s.shape[0]):
+        L = int(lens[r])
+        ref = O.causal_topk_row(s[r, :L].double().numpy(), L - 1, k)
+        errs = checks.topk_exact_errors(idx[r], ref, L - 1, k)
+        assert not errs, (r, errs[:3])
+        m = min(k, L)
+        assert np.array_equal(val[r, :m], s[r, idx[r, :m]].numpy() + 0.0)
+
+
+@pytest.mark.parametrize("k", [512, 2048])
+def test_topk_rows_long_rows_sample_prefilter(k):
+    """Rows of 8192..65536 entries take the sampled cut-off and the gather into
+    shared memory; rows of an odd width start off the 16-byte grid (head and
+    tail entries).  The result is the exact top-k."""
+    g = torch.Generator().manual_seed(100 + k)
+    rows, ncols = 8, 65543
+    s = torch.randn((rows, ncols), generator=g)
+    s[1] += torch.linspace(-3, 3, ncols)                   # a positional trend
+    s[2] = torch.randn(ncols, generator=g).exp()           # skewed
+    s[3, -3:] = 50.0                                       # the largest in the tail
+    s[4, :3] = 50.0                                        # ... and in the head
+    lens = torch.tensor([ncols, 65536, 40001, ncols, 20000, 8192, 8191, 4 * k + 1], dtype=torch.int32)
+    _topk_rows_check(s, lens, k)
+
+
+@pytest.mark.parametrize("k", [512, 2048])
+def test_topk_rows_long_rows_prefilter_fallbacks(k):
+    """Rows on which the sampled cut-off cannot work and the two-pass path
+    takes over: the sampled entries (every 16th group of four in a 16-byte
+    aligned row of 65536) hold the largest values, so fewer than k entries
+    reach the cut-off; all entries equal; four distinct values (the gathered
+    candidates overflow shared memory); a 0/1 row whose 1s are fewer than k."""
+    g = torch.Generator().manual_seed(200 + k)
+    rows, ncols = 5, 65536
+    s = torch.randn((rows, ncols), generator=g)
+    samp = (torch.arange(ncols) // 4) % 16 == 0
+    s[0, samp] += 100.0
+    s[1] = 0.25
+    s[2] = torch.randint(0, 4, (ncols,), generator=g).float()
+    s[3] = 0.0
+    s[3, torch.randperm(ncols, generator=g)[: k // 2]] = 1.0
+    s[4, samp] = 7.0
+    lens = torch.full((rows,), ncols, dtype=torch.int32)
+    _topk_rows_check(s, lens, k)
+
+
 # --------------------------------------------------------------------------
 # eqs. (1)+(2) fused, prefill
 # --------------------------------------------------------------------------
@@ -158,6 +210,38 @@ def test_prefill_tiny_exact():
 def test_prefill_integer_exact_ragged(HI, dI, n, k):
     w = W.scaled(W.PREFILL, B=2, n=n, HI=HI, dI=dI, k=k, seed=HI + n)
     _prefill_exact(w)
+
+
+def test_prefill_bounded_workspace_second_pass():
+    """History past 16384 keys with the bounded workspace: keys with equal
+    scores everywhere but at 300 raised positions, so every token accepts its
+    whole history and overflows its candidate buffer; 256 rows (four batches
+    of the second pass) are recomputed and selected exactly: the raised keys
+    up to t, then the lowest positions (eq. (2), ties to the lower position).
+    The full-history workspace (no second pass) gives the same indices."""
+    g = torch.Generator().manual_seed(31)
+    B, kv, nq, HI, dI, k = 1, 20480, 256, 8, 64, 2048
+    q0 = kv - nq
+    base = torch.randint(-2, 3, (dI,), generator=g).float()
+    kI = base.repeat(B, kv, 1)
+    raised = torch.randperm(kv, generator=g)[:300]
+    kI[0, raised] = 2 * base
+    qI = base.repeat(B, nq, HI, 1) + torch.randint(0, 2, (B, nq, HI, dI), generator=g).float()
+    w = torch.randint(1, 16, (B, nq, HI), generator=g).float() / 16
+    qd, kd, wd = qI.bfloat16().cuda(), kI.bfloat16().cuda(), w.cuda()
+    ws = _ws()
+    idx = dsa.indexer_topk_prefill(qd, kd, wd, k, q_offset=q0, workspace=ws)
+    full = dsa.indexer_topk_prefill(qd, kd, wd, k, q_offset=q0, workspace=ws, full_workspace=True)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    assert torch.equal(idx.sort(-1).values, full.sort(-1).values)     # slot order is unspecified
+    rows = [(0, i) for i in range(0, nq, 5)] + [(0, nq - 1)]
+    ref = O.indexer_topk(qI.double().numpy(), kI.double().numpy(), w.double().numpy(), k, q_offset=q0, rows=rows)
+    idx = idx.cpu().numpy()
+    bad = []
+    for b, i in rows:
+        bad += checks.topk_exact_errors(idx[b, i], ref[b, i], q0 + i, k)
+    assert not bad, bad[:5]
 
 
 def test_prefill_chunked_equals_whole():
