@@ -49,6 +49,7 @@ import torch  # noqa: E402
 from learned_token_indexer_b200 import workloads as W  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20
+LONG_STEP_MS = 50.0   # steps at least this long time their kernels at the sustained clock
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 METRIC = {
     "prefill": ("prefill query-tokens/s (indexer+top-k+sparse attn)", "query-tokens/s"),
@@ -828,6 +829,10 @@ def measure_workload(w, args, dev, world, rank, local, steps, warmup, cpu_budget
     if rank != 0:
         return None
     peaks, peak_src = load_peaks()
+    # a kernel timed inside a long step runs at the power-capped clock: its
+    # tensor peak is the sustained figure, the burst one for a short step
+    long_step = ms >= LONG_STEP_MS and "bf16_tflops_sustained" in peaks
+    tensor_peak = peaks["bf16_tflops_sustained"] if long_step else peaks["bf16_tflops"]
     names = list(work.keys())
     kernels = {}
     for name, wk in work.items():
@@ -839,7 +844,7 @@ def measure_workload(w, args, dev, world, rank, local, steps, warmup, cpu_budget
             per_launch = wk["flops"] / per_step_launches
             # a contraction takes the peak of its own dtype: e4m3 = the
             # measured bf16 figure x the nominal fp8 / bf16 ratio (2)
-            peak = peaks["bf16_tflops"] * (2.0 if fp8_mma else 1.0)
+            peak = tensor_peak * (2.0 if fp8_mma else 1.0)
             ach = per_launch / (t_launch * 1e-3) / 1e12
             bound = "tensor"
         else:
@@ -854,8 +859,13 @@ def measure_workload(w, args, dev, world, rank, local, steps, warmup, cpu_budget
                          "frac": round(ach / peak, 4), "ms_per_launch": round(t_launch, 4),
                          "traffic": measured_traffic(tkey, twl),
                          "algorithmic_per_launch": per_launch, "per_unit": wk["per_unit"]}
+        if bound == "tensor":
+            kernels[name]["peak_source"] = (
+                f"sustained bf16 ({peaks['bf16_tflops_sustained']} TFLOP/s: timed inside a {ms:.0f} ms step)"
+                if long_step else "burst bf16")
+            kernels[name]["frac_of_burst"] = round(ach / (peaks["bf16_tflops"] * (2.0 if fp8_mma else 1.0)), 4)
         if fp8_mma:
-            kernels[name]["peak_source"] = "fp8 = 2 x measured bf16 (nominal ratio)"
+            kernels[name]["peak_source"] += "; fp8 = 2 x that bf16 figure (nominal ratio)"
             if fp8_peak and fp8_peak.get("tflops"):
                 kernels[name]["fp8_peak_measured"] = dict(fp8_peak)
                 kernels[name]["frac_of_measured_fp8"] = round(ach / fp8_peak["tflops"], 4)
@@ -868,7 +878,9 @@ def measure_workload(w, args, dev, world, rank, local, steps, warmup, cpu_budget
     roof = {k: kernels[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roof["kernel"] = dom
     roof["peak_source"] = (f"{peak_src} "
-                           f"({kernels[dom].get('peak_source', 'burst bf16 / copy bandwidth')}; of measured)")
+                           f"({kernels[dom].get('peak_source', 'copy bandwidth')}; of {peak_src})")
+    if "frac_of_burst" in kernels[dom]:
+        roof["frac_of_burst"] = kernels[dom]["frac_of_burst"]
     metric, unit = METRIC[w.kind]
     rec = {
         "metric": metric, "value": job_throughput(world, rows, ms), "unit": unit,

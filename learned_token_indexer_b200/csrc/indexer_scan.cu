@@ -8,7 +8,8 @@
 //
 // Per CTA: warp 0 = TMA producer, warp 1 = tcgen05 MMA issuer (and TMEM
 // owner), warps 2..9 = two epilogue warpgroups (TMEM -> ReLU * w -> head sum
-// -> global).  The MMA computes D[128 keys x N] with keys on TMEM lanes and
+// -> global); with an e4m3 cache, warp 10 stages each tile's per-key scales
+// into a shared ring by cp.async, so no epilogue thread waits on them.  The MMA computes D[128 keys x N] with keys on TMEM lanes and
 // the token's heads on columns into four accumulators used in turn; the two
 // warpgroups take alternate tiles, so two tiles' epilogues run at once while
 // the MMA fills the next ones.  Work items are (row, run of key tiles),
@@ -21,15 +22,19 @@ namespace dsa {
 
 namespace {
 
-// K tiles in flight: 128 KB of K^I per CTA whatever the tile size (a 128-byte
-// row tile, e4m3 or d^I = 64 bf16, needs twice as many tiles in flight as a
-// 256-byte one to keep the same bytes on the way from HBM).
+// K tiles in flight: as many as shared memory holds beside the q tiles and
+// the row prefix (11 tiles of 128-byte rows = 176 KB, 5 of 256-byte rows =
+// 160 KB).  Under the scan's load the HBM latency is 2.5-4.5 us, so the bytes
+// in flight per SM set the rate (a tile every 0.54 us with 128 KB in flight).
 template <int KB>
-constexpr int scan_stages() { return KB == 1 ? 8 : 4; }
-constexpr int kScanThreads = 320;
+constexpr int scan_stages() { return KB == 1 ? 11 : 5; }
 constexpr int kEpiWarp0 = 2;
 constexpr int kEpiWarps = 8;     // two warpgroups
+constexpr int kScaleWarp = kEpiWarp0 + kEpiWarps;   // e4m3 only
 constexpr int kScanAcc = 4;      // accumulators in TMEM
+constexpr int kScaleStages = 8;  // tiles of key scales in flight
+template <bool FP8>
+constexpr int scan_threads() { return 32 * (kScaleWarp + (FP8 ? 1 : 0)); }
 
 struct ScanRow {
   int64_t key_base;
@@ -107,7 +112,7 @@ __device__ __forceinline__ float scan_head_sum(const uint32_t (&acc)[HI], const 
 }  // namespace
 
 template <int HI, bool FP8, int KB>
-__global__ void __launch_bounds__(kScanThreads, 1)
+__global__ void __launch_bounds__(scan_threads<FP8>(), 1)
     indexer_scan_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                         const ScanArgs a) {
   constexpr int N = HI < 16 ? 16 : HI;
@@ -134,7 +139,10 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   uint64_t* acc_full = q_empty + 2;
   uint64_t* acc_empty = acc_full + kScanAcc;
   uint64_t* mma_done = acc_empty + kScanAcc;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* ks_full = mma_done + 1;                 // [kScaleStages] (e4m3)
+  uint64_t* ks_empty = ks_full + kScaleStages;      // [kScaleStages]
+  float* sKS = reinterpret_cast<float*>(ks_empty + kScaleStages);   // [kScaleStages][128]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sKS + kScaleStages * kTileKeys);
   volatile uint32_t* abort_flag = tmem_slot + 1;
   int* sPre = reinterpret_cast<int*>(tmem_slot + 4);   // [rows + 1] in balanced mode
 
@@ -153,6 +161,10 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       mbar_init(&acc_empty[s], 4);              // the four warps of the warpgroup that reads it
     }
     mbar_init(mma_done, 1);
+    for (int s = 0; s < kScaleStages; ++s) {
+      mbar_init(&ks_full[s], 32);   // one cp.async arrival per lane of the scale warp
+      mbar_init(&ks_empty[s], 4);   // the four warps of the warpgroup that reads the tile
+    }
     *abort_flag = 0u;
     mbar_fence_init();
   }
@@ -167,7 +179,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   // balanced numbering needs the ragged offsets and room for the prefix
   const bool balanced = a.balanced != 0 && a.mode == 1 && a.rows <= kScanMaxBalancedRows;
   if (balanced) {
-    for (int r = threadIdx.x; r < a.rows; r += kScanThreads) {
+    for (int r = threadIdx.x; r < a.rows; r += scan_threads<FP8>()) {
       const int64_t len = a.cu_seqlens[r + 1] - a.cu_seqlens[r];
       const int tiles = (int)((len + kTileKeys - 1) / kTileKeys);
       sPre[r + 1] = (tiles + a.chunk_tiles - 1) / a.chunk_tiles;
@@ -200,6 +212,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      // K^I is read once: evicted from L2 first, so the scores stay there
+      const uint64_t k_policy = l2_policy_evict_first();
       int stage = 0, qslot = 0;
       uint32_t kphase = 0, qphase = 0;
       uint32_t k_last_parity[kScanStages], q_last_parity[2];
@@ -226,8 +240,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           mbar_arrive_expect_tx(&k_full[stage], kKBytes);
           const int y = (int)(g.key_base + (int64_t)(t0 + t) * kTileKeys);
           for (int kb = 0; kb < KB; ++kb)
-            tma_load_2d(sK + stage * kKBytes + kb * kTileKeys * kSwizzleBytes, &tmap_k, &k_full[stage],
-                        kb * kElemsPerBlock, y);
+            tma_load_2d_hint(sK + stage * kKBytes + kb * kTileKeys * kSwizzleBytes, &tmap_k, &k_full[stage],
+                             kb * kElemsPerBlock, y, k_policy);
           k_issued[stage] = true;
           k_last_parity[stage] = kphase;
           if (++stage == kScanStages) { stage = 0; kphase ^= 1u; }
@@ -288,11 +302,38 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       }
     }
     __syncwarp();
+  } else if (FP8 && warp == (uint32_t)kScaleWarp) {
+    // ------------------------------------------------------------ key scales (e4m3)
+    // Tile n's 128 scales go to ring slot n % kScaleStages; lane l copies
+    // keys l, l + 32, l + 64, l + 96 and its arrival fires when they land.
+    uint32_t n = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
+      int row, t0, nt;
+      ScanRow gr;
+      scan_item(a, item, row, t0, nt, gr, sPre, balanced);
+      for (int t = 0; t < nt; ++t, ++n) {
+        const uint32_t ks = n % kScaleStages;
+        const bool got = mbar_wait(&ks_empty[ks], ((n / kScaleStages) & 1u) ^ 1u, ctl, 0x401);
+        if (!(ok = __all_sync(0xffffffffu, got))) break;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int key = (t0 + t) * kTileKeys + 32 * j + (int)lane;
+          const bool in = key < gr.len;
+          cp_async_4(smem_u32(sKS + ks * kTileKeys + 32 * j + lane), in ? a.k_scale + gr.key_base + key : a.k_scale,
+                     in ? 4u : 0u);
+        }
+        cp_async_arrive_noinc(&ks_full[ks]);
+      }
+    }
+    cp_async_wait_all();   // nothing may land after the CTA is gone
   } else {
     // ------------------------------------------------------------ epilogue
     // Same barrier sequence for every thread; a failed wait only disables work.
     // Warpgroup g takes the tiles whose sequence number n has n % 2 == g.
     const uint32_t g = (warp - kEpiWarp0) >> 2;       // 0..1
+    // the scores are read again by the row top-k right after: kept in L2
+    const uint64_t out_policy = l2_policy_evict_last();
     const uint32_t lane_grp = (warp & 3u) * 32u;      // TMEM lanes this warp may access
     int qslot = 0;
     uint32_t qphase = 0, n = 0;
@@ -311,10 +352,16 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         if ((n & 1u) != g) continue;
         const uint32_t acc = n % kScanAcc, aphase = (n / kScanAcc) & 1u;
         const int s = (t0 + t) * kTileKeys + (int)lane_grp + (int)lane;
-        // the key's FP8 scale is requested before the wait, so its latency
-        // hides behind the MMA instead of following the head sum
         float kscale = 1.0f;
-        if (FP8 && s < gr.len) kscale = __ldg(a.k_scale + gr.key_base + s) * qs;
+        if constexpr (FP8) {
+          // the key's scale, staged by the scale warp
+          const uint32_t ks = n % kScaleStages;
+          const bool gs = ok && mbar_wait(&ks_full[ks], (n / kScaleStages) & 1u, ctl, 0x302);
+          ok = __all_sync(0xffffffffu, gs);
+          kscale = sKS[ks * kTileKeys + lane_grp + lane] * qs;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ks_empty[ks]);
+        }
         const bool got = ok && mbar_wait(&acc_full[acc], aphase, ctl, 0x301);
         ok = __all_sync(0xffffffffu, got);
         if (ok) {
@@ -328,7 +375,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           if (s < gr.len) {
             float score = scan_head_sum<HI>(r, w_row);
             if (FP8) score *= kscale;
-            gr.out[s] = score + 0.0f;
+            st_global_hint(gr.out + s, score + 0.0f, out_policy);
           }
         }
       }
@@ -350,7 +397,8 @@ template <int HI, bool FP8, int KB>
 static size_t scan_smem_bytes() {
   constexpr int N = HI < 16 ? 16 : HI;
   return 1024 + scan_stages<KB>() * kTileKeys * KB * kSwizzleBytes + 2 * N * KB * kSwizzleBytes + 2 * HI * 4 +
-         (2 * scan_stages<KB>() + 4 + 2 * kScanAcc + 1) * 8 + 16 + (kScanMaxBalancedRows + 1) * 4;
+         (2 * scan_stages<KB>() + 4 + 2 * kScanAcc + 1 + 2 * kScaleStages) * 8 + kScaleStages * kTileKeys * 4 + 16 +
+         (kScanMaxBalancedRows + 1) * 4;
 }
 
 template <int HI, bool FP8, int KB>
@@ -360,7 +408,7 @@ static cudaError_t launch_scan_t(const CUtensorMap& tq, const CUtensorMap& tk, c
   auto kern = indexer_scan_kernel<HI, FP8, KB>;
   cudaError_t e = setup_once_per_device([&]() { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); });
   if (e != cudaSuccess) return e;
-  kern<<<grid, kScanThreads, smem, stream>>>(tq, tk, a);
+  kern<<<grid, scan_threads<FP8>(), smem, stream>>>(tq, tk, a);
   return cudaGetLastError();
 }
 

@@ -390,12 +390,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             if (lane == (uint32_t)(__ffs(peers) - 1)) atomicAdd(&sHist[st * kHistBins + bin], (uint32_t)__popc(peers));
           }
           cnt[u] += (uint32_t)__popc(mask);
-          // raise the floor (every tile, by a warp that rotates with the
-          // tile so the four warps share the work): the bin where the count
-          // of accepted scores from the top first reaches k.  Two warps may
-          // raise one token's floor at once; each value written is a valid
-          // floor (counts only grow), so a lost update only admits more
-          if (quarter == ((uint32_t)(t + 2 * u) & 3u))
+          // raise the floor (every tile for the first 64 tiles, then on 4
+          // tiles of every 16, where a long history has settled it; by a
+          // warp that rotates with the tile so the four warps share the
+          // work): the bin where the count of accepted scores from the top
+          // first reaches k.  Two warps may raise one token's floor at once;
+          // each value written is a valid floor (counts only grow), so a lost
+          // update only admits more
+          if (quarter == ((uint32_t)(t + 2 * u) & 3u) && (t < 64 || ((t >> 2) & 3) == 0))
             raise_floor(sHist + st * kHistBins, (uint32_t)a.k, &sFloorKey[st], lane);
         }
       }

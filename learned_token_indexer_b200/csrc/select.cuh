@@ -99,8 +99,23 @@ __device__ __forceinline__ bool group_find(const uint32_t* hist, int nbins, uint
   }
   if (lane == 31) sh.warp_sum[w] = incl;
   named_bar_sync(bar_id, NT);
-  uint32_t before = incl - local;
-  for (uint32_t j = 0; j < w; ++j) before += sh.warp_sum[j];
+  // entries in the warps before this one: a scan over the warp sums
+  // (a loop over them would be a chain of up to 31 shared loads)
+  constexpr int NW = NT / 32;
+  uint32_t wpre = 0;
+  if constexpr (NW <= 4) {
+    for (uint32_t j = 0; j < w; ++j) wpre += sh.warp_sum[j];
+  } else {
+    const uint32_t v = lane < (uint32_t)NW ? sh.warp_sum[lane] : 0u;
+    uint32_t sc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, sc, o);
+      if (lane >= (uint32_t)o) sc += t;
+    }
+    wpre = __shfl_sync(0xffffffffu, sc - v, w);
+  }
+  uint32_t before = incl - local + wpre;
   if (before < need && need <= before + local) {
     uint32_t run = before;
     for (int i = i0; i < i0 + per && i < nbins; ++i) {

@@ -26,9 +26,10 @@ namespace dsa {
 namespace {
 constexpr int kRowThreads = 1024;
 constexpr int kRowBins = 2048;        // refinement digit bins
-constexpr int kBndCap = 4096;         // cut-off bin entries kept in shared memory (two-pass path)
+constexpr int kBndCap = 16384;        // cut-off bin entries kept in shared memory (two-pass path)
 constexpr int kCandCap = 16384;       // gathered candidates (prefilter path)
 constexpr int kSampleMax = 8192;      // sampled entries
+constexpr int kSampleLong = 1024;     // sampled entries of a row of at least 16384
 constexpr int kGatherBatch = 4;       // 16-byte loads in flight per thread in the gather pass
 constexpr int kPrefilterMinLen = 8192;
 constexpr size_t kTopkDynSmem = (size_t)kCandCap * sizeof(uint2);
@@ -38,6 +39,7 @@ static_assert(kBndCap <= kCandCap && kSampleMax * sizeof(uint32_t) <= kTopkDynSm
 __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRowsArgs a) {
   __shared__ uint32_t hist[kRowBins];
   __shared__ SelectShared<kRowThreads> sh;
+  __shared__ uint32_t s_maxkey;   // largest key of the row (prefilter path)
   extern __shared__ __align__(16) uint8_t topk_dyn[];
   uint2* cand = reinterpret_cast<uint2*>(topk_dyn);     // prefilter candidates
   uint32_t* samp = reinterpret_cast<uint32_t*>(topk_dyn);  // sample keys (before the gather)
@@ -81,9 +83,18 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRow
   // ---- prefilter for long rows
   const int head = min(len, (int)((((16u - ((uint32_t)reinterpret_cast<uintptr_t>(src) & 15u)) & 15u)) >> 2));
   const int nb4 = (len - head) >> 2;                    // 16-byte aligned body, in float4
+  const float4* body = reinterpret_cast<const float4*>(src + head);
   if (len >= kPrefilterMinLen && len >= 4 * kk) {
-    const float4* body = reinterpret_cast<const float4*>(src + head);
-    const int ns4 = min(nb4 >> 4, kSampleMax / 4);
+    // the row is pulled into L2 now, for the gather pass after the sample
+    if (tid < 32) {
+      constexpr int64_t kChunk = 65536;
+      const int64_t bytes = (int64_t)nb4 * 16;
+      for (int64_t o = (int64_t)tid * kChunk; o < bytes; o += 32 * kChunk)
+        prefetch_l2_bulk(reinterpret_cast<const char*>(body) + o, (uint32_t)min(kChunk, bytes - o));
+    }
+    if (tid == 0) s_maxkey = 0u;
+    // 1024 sampled entries for long rows (1/16 of shorter ones)
+    const int ns4 = nb4 >= 16 * (kSampleLong / 4) ? kSampleLong / 4 : min(nb4 >> 4, kSampleMax / 4);
     const int st = nb4 / ns4;                            // >= 16
     const int s_n = 4 * ns4;
     for (int j = (int)tid; j < ns4; j += kRowThreads) {
@@ -94,16 +105,18 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRow
       samp[4 * j + 3] = float_to_key(v.w);
     }
     __syncthreads();
-    // m-th largest sampled key, m about 1.25 kk s/len plus a margin, so that
-    // more than kk row entries reach it unless the sample is unrepresentative
+    // tau = the lower edge of the top-11-bit key bin holding the m-th largest
+    // sampled key, m about 1.25 kk s/len plus a margin, so that more than kk
+    // row entries reach it unless the sample is unrepresentative (one
+    // histogram round: the exact select runs on the gathered entries)
     const int m = (int)((5LL * kk * s_n + 4LL * len - 1) / (4LL * len)) + 32;
-    auto get_s = [samp](int i, uint32_t& key, uint32_t& pos) {
-      key = samp[i];
-      pos = (uint32_t)i;
-    };
-    const SelectResult rs = group_refine<kRowThreads, kRowBins>(get_s, s_n, 0u, 0xFFFFFFFFu, (uint32_t)m,
-                                                                (uint32_t)(s_n - 1), hist, sh, tid, 0, a.status);
-    const uint32_t tau = rs.lo;
+    for (int i = (int)tid; i < kRowBins; i += kRowThreads) hist[i] = 0u;
+    __syncthreads();
+    for (int j = (int)tid; j < s_n; j += kRowThreads) atomicAdd(&hist[samp[j] >> 21], 1u);
+    __syncthreads();
+    if (!group_find<kRowThreads>(hist, kRowBins, (uint32_t)m, true, sh, tid, 0) && tid == 0)
+      report_status(a.status, kStatusDeviceCheck, 0x5e1ecau);
+    const uint32_t tau = sh.found_bin << 21;
     if (tid == 0) sh.bnd_count = 0u;
     __syncthreads();   // sample reads done before the buffer is reused
     for (int j0 = 0; j0 < nb4; j0 += kRowThreads * kGatherBatch) {
@@ -113,14 +126,19 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRow
         const int j = j0 + u * kRowThreads + (int)tid;
         v[u] = j < nb4 ? body[j] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      uint32_t n = 0;
+      uint32_t n = 0, kmax = 0;
 #pragma unroll
       for (int u = 0; u < kGatherBatch; ++u) {
         const int j = j0 + u * kRowThreads + (int)tid;
-        if (j < nb4)
-          n += (float_to_key(v[u].x) >= tau) + (float_to_key(v[u].y) >= tau) + (float_to_key(v[u].z) >= tau) +
-               (float_to_key(v[u].w) >= tau);
+        if (j < nb4) {
+          const uint32_t k0 = float_to_key(v[u].x), k1 = float_to_key(v[u].y), k2 = float_to_key(v[u].z),
+                         k3 = float_to_key(v[u].w);
+          n += (k0 >= tau) + (k1 >= tau) + (k2 >= tau) + (k3 >= tau);
+          kmax = max(kmax, max(max(k0, k1), max(k2, k3)));
+        }
       }
+      kmax = __reduce_max_sync(0xffffffffu, kmax);
+      if (lane == 0) atomicMax(&s_maxkey, kmax);
       uint32_t incl = n;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -152,6 +170,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRow
       const bool valid = tid < 3 ? i < head : (tid < 6 && i < len);
       const uint32_t key = valid ? float_to_key(src[i]) : 0u;
       const bool take = valid && key >= tau;
+      if (take) atomicMax(&s_maxkey, key);
       const uint32_t mk = __ballot_sync(0xffffffffu, take);
       uint32_t base = 0;
       if (lane == 0 && mk) base = atomicAdd(&sh.bnd_count, (uint32_t)__popc(mk));
@@ -162,7 +181,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRow
       }
     }
     __syncthreads();
-    const uint32_t c = sh.bnd_count;
+    const uint32_t c = sh.bnd_count, kmax = s_maxkey;
     __syncthreads();   // every thread has read the count before the select reuses sh
     if (c >= (uint32_t)kk && c <= (uint32_t)kCandCap) {
       auto get_c = [cand](int i, uint32_t& key, uint32_t& pos) {
@@ -170,7 +189,8 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRow
         key = e.x;
         pos = e.y;
       };
-      const SelectResult r = group_refine<kRowThreads, kRowBins>(get_c, (int)c, tau, 0xFFFFFFFFu, (uint32_t)kk,
+      // every candidate key lies in [tau, kmax]
+      const SelectResult r = group_refine<kRowThreads, kRowBins>(get_c, (int)c, tau, max(tau, kmax), (uint32_t)kk,
                                                                  (uint32_t)(len - 1), hist, sh, tid, 0, a.status);
       group_emit<kRowThreads>(get_c, (int)c, r, kk, a.k, idx_row, val_row, sh, tid, 0, a.status);
       return;
@@ -207,38 +227,97 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_rows_kernel(const TopkRow
     sh.bnd_count = 0u;
   }
   __syncthreads();
-  for (int j0 = 0; j0 < len; j0 += kRowThreads * kBatch) {
-    uint32_t key[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int i = j0 + u * kRowThreads + (int)tid;
-      key[u] = i < len ? float_to_key(src[i]) : 0u;
+  // one entry per thread (all lanes of the warp take part): above the
+  // cut-off bin -> written to the output now; inside it -> shared memory
+  auto classify = [&](bool valid, uint32_t key, int i) {
+    const bool above = valid && key > bhi, on = valid && key >= blo && key <= bhi;
+    const uint32_t ma = __ballot_sync(0xffffffffu, above), mo = __ballot_sync(0xffffffffu, on);
+    uint32_t base_a = 0, base_o = 0;
+    if (lane == 0) {
+      if (ma) base_a = atomicAdd(&sh.out_count, (uint32_t)__popc(ma));
+      if (mo) base_o = atomicAdd(&sh.bnd_count, (uint32_t)__popc(mo));
     }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int i = j0 + u * kRowThreads + (int)tid;
-      const bool above = i < len && key[u] > bhi, on = i < len && key[u] >= blo && key[u] <= bhi;
-      const uint32_t ma = __ballot_sync(0xffffffffu, above), mo = __ballot_sync(0xffffffffu, on);
-      uint32_t base_a = 0, base_o = 0;
-      if (lane == 0) {
-        if (ma) base_a = atomicAdd(&sh.out_count, (uint32_t)__popc(ma));
-        if (mo) base_o = atomicAdd(&sh.bnd_count, (uint32_t)__popc(mo));
+    base_a = __shfl_sync(0xffffffffu, base_a, 0);
+    base_o = __shfl_sync(0xffffffffu, base_o, 0);
+    const uint32_t below = (1u << lane) - 1u;
+    if (above) {
+      const uint32_t slot = base_a + __popc(ma & below);
+      if (slot < (uint32_t)kk) {
+        idx_row[slot] = i;
+        if (val_row) val_row[slot] = key_to_float(key);
       }
-      base_a = __shfl_sync(0xffffffffu, base_a, 0);
-      base_o = __shfl_sync(0xffffffffu, base_o, 0);
-      const uint32_t below = (1u << lane) - 1u;
-      if (above) {
-        const uint32_t slot = base_a + __popc(ma & below);
-        if (slot < (uint32_t)kk) {
-          idx_row[slot] = i;
-          if (val_row) val_row[slot] = key_to_float(key[u]);
+    }
+    if (on) {
+      const uint32_t slot = base_o + __popc(mo & below);
+      if (slot < (uint32_t)kBndCap) bnd[slot] = make_uint2(key, (uint32_t)i);
+    }
+  };
+  // the 16-byte aligned body with 16-byte loads, then the head and tail;
+  // per thread and batch of 16 entries: both counts, one warp scan of the
+  // packed pair and one pair of shared atomics per warp
+  for (int j0 = 0; j0 < nb4; j0 += kRowThreads * kGatherBatch) {
+    float4 v[kGatherBatch];
+#pragma unroll
+    for (int u = 0; u < kGatherBatch; ++u) {
+      const int j = j0 + u * kRowThreads + (int)tid;
+      v[u] = j < nb4 ? body[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    uint32_t na = 0, no = 0;
+#pragma unroll
+    for (int u = 0; u < kGatherBatch; ++u) {
+      const int j = j0 + u * kRowThreads + (int)tid;
+      if (j < nb4) {
+        const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t key = float_to_key(f[c]);
+          na += key > bhi;
+          no += key >= blo && key <= bhi;
         }
       }
-      if (on) {
-        const uint32_t slot = base_o + __popc(mo & below);
-        if (slot < (uint32_t)kBndCap) bnd[slot] = make_uint2(key[u], (uint32_t)i);
+    }
+    const uint32_t packed = na | (no << 16);   // each count <= 16 per thread, <= 512 per warp
+    uint32_t incl = packed;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= (uint32_t)o) incl += t;
+    }
+    uint32_t base_a = 0, base_o = 0;
+    if (lane == 31) {
+      if (incl & 0xFFFFu) base_a = atomicAdd(&sh.out_count, incl & 0xFFFFu);
+      if (incl >> 16) base_o = atomicAdd(&sh.bnd_count, incl >> 16);
+    }
+    const uint32_t excl = incl - packed;
+    uint32_t pa = __shfl_sync(0xffffffffu, base_a, 31) + (excl & 0xFFFFu);
+    uint32_t po = __shfl_sync(0xffffffffu, base_o, 31) + (excl >> 16);
+    if (na | no) {
+#pragma unroll
+      for (int u = 0; u < kGatherBatch; ++u) {
+        const int j = j0 + u * kRowThreads + (int)tid;
+        const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t key = float_to_key(f[c]);
+          if (j < nb4 && key > bhi) {
+            if (pa < (uint32_t)kk) {
+              idx_row[pa] = head + 4 * j + c;
+              if (val_row) val_row[pa] = key_to_float(key);
+            }
+            ++pa;
+          } else if (j < nb4 && key >= blo) {
+            if (po < (uint32_t)kBndCap) bnd[po] = make_uint2(key, (uint32_t)(head + 4 * j + c));
+            ++po;
+          }
+        }
       }
     }
+  }
+  if (tid < 32) {
+    const int tail0 = head + 4 * nb4;
+    const int i = tid < 3 ? (int)tid : tail0 + (int)tid - 3;
+    const bool valid = tid < 3 ? i < head : (tid < 6 && i < len);
+    classify(valid, valid ? float_to_key(src[i]) : 0u, i);
   }
   __syncthreads();
   const uint32_t nb = sh.bnd_count;

@@ -446,6 +446,37 @@ def test_decode_fp8_cache_small_ragged():
     _decode_case(w, torch.tensor([1, 129, 300, 1000, 4097]))
 
 
+def test_decode_selection_with_equal_scores():
+    """Decode selection on caches whose keys mostly repeat one vector, so the
+    scan's histogram puts whole sequences into one cut-off bin: more entries
+    than shared memory holds for the longest (the refinement then runs over
+    the row), a sequence whose raised keys all fit, and short ones.  Integer
+    values: the selection is exact (equal scores go to the lower position)."""
+    g = torch.Generator().manual_seed(41)
+    lengths = torch.tensor([40000, 20000, 2100, 5])
+    B, HI, dI, k = lengths.numel(), 16, 64, 2048
+    cu = torch.zeros(B + 1, dtype=torch.int64)
+    cu[1:] = torch.cumsum(lengths, 0)
+    total = int(cu[-1])
+    base = torch.randint(-2, 3, (dI,), generator=g).float()
+    kc = base.repeat(total, 1)
+    raised = torch.randperm(total, generator=g)[:700]
+    kc[raised] = 2 * base
+    q = base.repeat(B, HI, 1) + torch.randint(0, 2, (B, HI, dI), generator=g).float()
+    w = torch.randint(1, 16, (B, HI), generator=g).float() / 16
+    ws = _ws()
+    idx = dsa.indexer_topk_decode(q.bfloat16().cuda(), w.cuda(), kc.bfloat16().cuda(), cu.cuda(), k, total,
+                                  int(lengths.max()), workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    ref = O.decode_indexer_topk(q.double().numpy(), w.double().numpy(), kc.double().numpy(), cu, k)
+    idx = idx.cpu().numpy()
+    bad = []
+    for b in range(B):
+        bad += checks.topk_exact_errors(idx[b], ref[b], int(lengths[b]) - 1, k)
+    assert not bad, bad[:5]
+
+
 def test_decode_attention_scattered_and_bad_slots():
     """The decode step's attention (128 heads, 576/512 latent rows: the
     tensor-core kernel whose two CTAs split the latent columns) on ragged
