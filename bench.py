@@ -562,6 +562,7 @@ def time_e2e_pipelined(runs, steps):
     overlap step i).  Every step still uploads its inputs from pinned host
     memory and downloads its result.  Returns ms per step (device events from
     the first upload to the last download)."""
+    assert len(runs) >= 2, "the next step's upload goes to the other replica"
     host = runs[0].host_inputs()
     shape, dtype = runs[0].result().shape, runs[0].result().dtype
     res_host = [torch.empty(shape, dtype=dtype, pin_memory=True) for _ in runs]
@@ -570,19 +571,29 @@ def time_e2e_pipelined(runs, steps):
     def go(n, start=None):
         done_run = [None] * len(runs)   # the replica's last step has consumed its inputs
         done_out = [None] * len(runs)   # the replica's last result has been read out
-        if start is not None:
-            start.record(s_in)
-        for i in range(n):
+        loaded = [None] * len(runs)     # the replica's inputs for its next step are in
+
+        def upload(i):
             j = i % len(runs)
-            r = runs[j]
             with torch.cuda.stream(s_in):
                 if done_run[j] is not None:
                     s_in.wait_event(done_run[j])
-                r.load_inputs(host)
-                loaded = torch.cuda.Event()
-                loaded.record(s_in)
+                runs[j].load_inputs(host)
+                loaded[j] = torch.cuda.Event()
+                loaded[j].record(s_in)
+
+        if start is not None:
+            start.record(s_in)
+        upload(0)
+        for i in range(n):
+            j = i % len(runs)
+            r = runs[j]
+            # the next step's upload is queued before this step, so it overlaps
+            # the step even when a call inside the step waits on the host
+            if i + 1 < n:
+                upload(i + 1)
             with torch.cuda.stream(s_run):
-                s_run.wait_event(loaded)
+                s_run.wait_event(loaded[j])
                 if done_out[j] is not None:
                     s_run.wait_event(done_out[j])
                 r.step()

@@ -251,7 +251,12 @@ size_t attn_teacher_smem_bytes(int k) { return (size_t)kTOffP + (size_t)k * 4; }
 
 cudaError_t launch_attn_teacher(const TeacherArgs& a, cudaStream_t stream) {
   const size_t smem = attn_teacher_smem_bytes(a.k);
-  cudaError_t e = setup_once_per_device([&]() { return cudaFuncSetAttribute(attn_teacher_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); });
+  // the attribute is an upper bound: set once for the largest k, so a later
+  // call with a larger k than the first still launches
+  cudaError_t e = setup_once_per_device([]() {
+    return cudaFuncSetAttribute(attn_teacher_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)attn_teacher_smem_bytes(kMaxTeacherTopk));
+  });
   if (e != cudaSuccess) return e;
   attn_teacher_kernel<<<a.rows, kTThreads, smem, stream>>>(a);
   return cudaGetLastError();

@@ -126,6 +126,33 @@ def test_prefill_workspace_is_bounded_past_16384_keys(lib):
     assert dec >= 256 + 4000
 
 
+def _decode(lib, **kw):
+    a = dict(B=2, HI=64, dI=128, k=8, dtype=0, q=16, qs=None, w=16, kc=16, ks=None, cu=16, total=100, maxlen=60,
+             idx=16, sc=None, ws=256, wsb=1 << 30)
+    a.update(kw)
+    p = lambda v: None if v is None else C.c_void_p(v)
+    return lib.dsa_indexer_topk_decode(a["B"], a["HI"], a["dI"], a["k"], a["dtype"], p(a["q"]), p(a["qs"]),
+                                       p(a["w"]), p(a["kc"]), p(a["ks"]), p(a["cu"]), a["total"], a["maxlen"],
+                                       p(a["idx"]), p(a["sc"]), p(a["ws"]), a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=0), 0),                  # an empty batch launches nothing
+    (dict(B=-1), 1),
+    (dict(k=0), 1),
+    (dict(HI=3), 2),
+    (dict(w=24), 1),                 # head weights are staged by a 16-byte bulk copy
+    (dict(q=8), 1),                  # misaligned TMA operand
+    (dict(kc=None), 1),
+    (dict(dtype=1, qs=None, ks=None), 1),
+    (dict(total=1 << 31), 2),        # cache rows past 2^31
+    (dict(wsb=64), 3),               # too small for the step's scores
+])
+def test_decode_argument_checks(lib, kw, status):
+    """Host checks of the decode step run before any launch (no GPU needed)."""
+    assert _decode(lib, **kw) == status
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "_lib", None)
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))

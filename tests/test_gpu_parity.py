@@ -244,6 +244,38 @@ def test_prefill_bounded_workspace_second_pass():
     assert not bad, bad[:5]
 
 
+def test_prefill_bounded_workspace_second_pass_fp8():
+    """The bounded workspace's second pass with an e4m3 indexer: identical
+    key rows get identical codes and scales (per-token quantisation), so the
+    scores tie exactly and the selection is exact; every row of the chunk
+    overflows and is recomputed by the e4m3 scan."""
+    g = torch.Generator().manual_seed(32)
+    B, kv, nq, HI, dI, k = 1, 18432, 160, 8, 64, 2048
+    q0 = kv - nq
+    base = torch.randn((dI,), generator=g)
+    kI = base.repeat(B, kv, 1)
+    raised = torch.randperm(kv, generator=g)[:200]
+    kI[0, raised] = 2 * base
+    qI = base.repeat(B, nq, HI, 1) + 0.25 * torch.randn((B, nq, HI, dI), generator=g)
+    w = torch.rand((B, nq, HI), generator=g) + 0.1
+    q8, qs = W.quantize_fp8_per_token(qI, 2)
+    k8, ks = W.quantize_fp8_per_token(kI, 1)
+    ws = _ws()
+    args = (q8.cuda(), k8.cuda(), w.cuda(), k)
+    idx = dsa.indexer_topk_prefill(*args, q_offset=q0, q_scale=qs.cuda(), k_scale=ks.cuda(), workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    qh, kh = host_dequant(q8, qs, 2), host_dequant(k8, ks, 1)
+    rows = [(0, i) for i in range(0, nq, 7)] + [(0, nq - 1)]
+    idx = idx.cpu().numpy()
+    bad = []
+    for b, i in rows:
+        sc = O.indexer_scores_row(qh[b, i], kh[b, : q0 + i + 1], w[b, i].double().numpy())
+        errs, _ = checks.topk_tolerant_errors(idx[b, i], sc, q0 + i, k)
+        bad += errs
+    assert not bad, bad[:5]
+
+
 def test_prefill_chunked_equals_whole():
     w = W.scaled(W.PREFILL, B=1, n=1536, k=200, seed=77)
     _prefill_exact(w, chunk=512)
@@ -406,7 +438,7 @@ def test_worked_example_through_the_library():
 # decode
 # --------------------------------------------------------------------------
 
-def _decode_case(w, lengths):
+def _decode_case(w, lengths, attention=True):
     d = W.make_decode_inputs(w, "cuda", lengths=lengths)
     total, maxlen = int(lengths.sum()), int(lengths.max())
     ws = _ws()
@@ -429,6 +461,8 @@ def _decode_case(w, lengths):
         errs, _ = checks.topk_tolerant_errors(idx_h[b], s, int(lengths[b]) - 1, w.k)
         bad += errs
     assert not bad, bad[:5]
+    if not attention:
+        return
     ro, rl = O.decode_sparse_attention(host_f64(d["q"]), host_f64(d["latent_cache"]), cu, idx_h, w.scale, w.Dv)
     bad = checks.close_errors(host_f64(out), ro, ATOL, RTOL, "decode out")
     bad += checks.close_errors(lse.cpu().double().numpy(), rl, 1e-3, 1e-3, "decode lse")
@@ -444,6 +478,15 @@ def test_decode_fp8_cache_small_ragged():
     # e4m3 K^I cache with one scale per key, e4m3 queries with one scale per token
     w = W.scaled(W.DECODE_FP8, B=5, k=300)
     _decode_case(w, torch.tensor([1, 129, 300, 1000, 4097]))
+
+
+def test_decode_lengths_around_the_selection_thresholds():
+    """Sequences at the row top-k's boundaries with k = 2048: t + 1 = k - 1,
+    k, k + 1 (everything / all but one selected), just below, at and above
+    the sampled cut-off's 8192-entry minimum, and around the 16384 entries
+    where the sample switches to 1024 entries."""
+    w = W.scaled(W.DECODE, k=2048)
+    _decode_case(w, torch.tensor([2047, 2048, 2049, 8191, 8192, 8193, 16383, 16384, 16389]), attention=False)
 
 
 def test_decode_selection_with_equal_scores():
