@@ -172,7 +172,7 @@ dsa_status dsa_attn_dense_prefill(int B, int nq, int q_offset, int kv_len, int H
 /* Length dispatch of the prefill attention (§2: the serving side picks the
  * path by length; masked dense attention wins for short histories).
  * dsa_prefill_attention_path returns DSA_PATH_DENSE_MASKED when the chunk's
- * longest history (q_offset + nq keys) is at most 4096 and the shape is the
+ * longest history (q_offset + nq keys) is at most 6144 and the shape is the
  * dense kernel's (H = 16, Dqk = 576, Dv = 512), else DSA_PATH_GATHER (the
  * threshold is where the two paths' measured times cross on one B200 with
  * k = 2048).  dsa_attn_prefill runs eq. (3) on that path with the arguments

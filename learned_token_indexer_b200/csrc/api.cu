@@ -467,10 +467,11 @@ dsa_status dsa_attn_dense_prefill(int B, int nq, int q_offset, int kv_len, int H
 
 // Length dispatch of the prefill attention (§2: short prefill runs DSA as
 // masked dense attention, long prefill gathers the selected rows).  Measured
-// on one B200 with k = 2048, 16 heads, 576/512 latent rows: the dense path
-// takes 0.25 / 0.88 / 3.20 ms for histories of 2048 / 4096 / 8192 keys, the
-// gathering path 0.40 / 1.05 / 2.36 ms.
-static constexpr int kDenseMaxHistory = 4096;
+// on one B200 with k = 2048, 16 heads, 576/512 latent rows, one sequence:
+// the dense path takes 0.77 / 1.16 / 1.65 / 2.20 / 2.82 ms for histories of
+// 4096 / 5120 / 6144 / 7168 / 8192 keys, the gathering path 1.04 / 1.36 /
+// 1.69 / 2.02 / 2.34 ms.
+static constexpr int kDenseMaxHistory = 6144;
 
 int dsa_prefill_attention_path(int B, int nq, int q_offset, int kv_len, int H, int Dqk, int Dv, int k) {
   (void)B;

@@ -241,44 +241,59 @@ __device__ __forceinline__ bool selected(const SelectResult& r, uint32_t key, ui
 
 // Write the selected entries (exactly kk of them) to idx_row[0..kk) in
 // unspecified order, scores too if score_row != nullptr, then pad [kk, k)
-// with -1 / -inf.
+// with -1 / -inf.  Output slots come from a group-wide scan of the per-warp
+// counts of each batch (two barriers a batch, no shared atomics).
 template <int NT, typename Get>
 __device__ void group_emit(Get get, int m, const SelectResult& r, int kk, int k, int32_t* idx_row,
                            float* score_row, SelectShared<NT>& sh, uint32_t tid, uint32_t bar_id,
                            DeviceStatus* status) {
-  if (tid == 0) sh.out_count = 0;
-  named_bar_sync(bar_id, NT);
-  const uint32_t lane = tid & 31u;
+  constexpr int NW = NT / 32;
+  const uint32_t lane = tid & 31u, w = tid >> 5;
+  uint32_t run = 0;
   for (int j0 = 0; j0 < m; j0 += NT * kBatch) {
     uint32_t key[kBatch], pos[kBatch];
+    uint32_t n = 0;
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       key[u] = 0u;
       pos[u] = 0u;
       const int i = j0 + u * NT + (int)tid;
       if (i < m) get(i, key[u], pos[u]);
+      n += (i < m && selected(r, key[u], pos[u])) ? 1u : 0u;
     }
+    uint32_t incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= (uint32_t)o) incl += t;
+    }
+    if (lane == 31) sh.warp_sum[w] = incl;
+    named_bar_sync(bar_id, NT);
+    const uint32_t tw = lane < (uint32_t)NW ? sh.warp_sum[lane] : 0u;
+    uint32_t sc = tw;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, sc, o);
+      if (lane >= (uint32_t)o) sc += t;
+    }
+    uint32_t slot = run + __shfl_sync(0xffffffffu, sc - tw, w) + incl - n;
+    run += __shfl_sync(0xffffffffu, sc, 31);
+    named_bar_sync(bar_id, NT);   // warp_sum is free for the next batch
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int i = j0 + u * NT + (int)tid;
-      const bool sel = i < m && selected(r, key[u], pos[u]);
-      const uint32_t mask = __ballot_sync(0xffffffffu, sel);
-      uint32_t base = 0;
-      if (lane == 0 && mask) base = atomicAdd(&sh.out_count, (uint32_t)__popc(mask));
-      base = __shfl_sync(0xffffffffu, base, 0);
-      if (sel) {
-        const uint32_t slot = base + __popc(mask & ((1u << lane) - 1u));
+      if (i < m && selected(r, key[u], pos[u])) {
         if (slot < (uint32_t)kk) {
           idx_row[slot] = (int32_t)pos[u];
           if (score_row) score_row[slot] = key_to_float(key[u]);
         }
+        ++slot;
       }
     }
   }
-  named_bar_sync(bar_id, NT);
   // A selection that does not produce exactly kk entries is a library bug:
   // report it and leave no stale slot behind.
-  const int got = (int)sh.out_count;
+  const int got = (int)run;
   if (got != kk && tid == 0) report_status(status, kStatusDeviceCheck, 0x5e1ec7u);
   for (int j = (got < kk ? got : kk) + (int)tid; j < k; j += NT) {
     idx_row[j] = -1;
@@ -289,38 +304,58 @@ __device__ void group_emit(Get get, int m, const SelectResult& r, int kk, int k,
 
 // Append the selected entries with keys in [key_lo, key_hi] among entries
 // [0, m) to idx_row / score_row at slots counted on from sh.out_count (which
-// the caller has set); no padding.
+// the caller has set and made visible with a barrier); no padding.  Slots
+// come from a group-wide scan of the per-warp counts of each batch.
 template <int NT, typename Get>
 __device__ void group_emit_append(Get get, int m, const SelectResult& r, uint32_t key_lo, uint32_t key_hi, int kk,
                                   int32_t* idx_row, float* score_row, SelectShared<NT>& sh, uint32_t tid,
                                   uint32_t bar_id) {
-  const uint32_t lane = tid & 31u;
+  constexpr int NW = NT / 32;
+  const uint32_t lane = tid & 31u, w = tid >> 5;
+  uint32_t run = sh.out_count;
   for (int j0 = 0; j0 < m; j0 += NT * kBatch) {
     uint32_t key[kBatch], pos[kBatch];
+    uint32_t n = 0;
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       key[u] = 0u;
       pos[u] = 0u;
       const int i = j0 + u * NT + (int)tid;
       if (i < m) get(i, key[u], pos[u]);
+      n += (i < m && key[u] >= key_lo && key[u] <= key_hi && selected(r, key[u], pos[u])) ? 1u : 0u;
     }
+    uint32_t incl = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= (uint32_t)o) incl += t;
+    }
+    if (lane == 31) sh.warp_sum[w] = incl;
+    named_bar_sync(bar_id, NT);
+    const uint32_t tw = lane < (uint32_t)NW ? sh.warp_sum[lane] : 0u;
+    uint32_t sc = tw;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, sc, o);
+      if (lane >= (uint32_t)o) sc += t;
+    }
+    uint32_t slot = run + __shfl_sync(0xffffffffu, sc - tw, w) + incl - n;
+    run += __shfl_sync(0xffffffffu, sc, 31);
+    named_bar_sync(bar_id, NT);   // warp_sum is free for the next batch
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int i = j0 + u * NT + (int)tid;
-      const bool sel = i < m && key[u] >= key_lo && key[u] <= key_hi && selected(r, key[u], pos[u]);
-      const uint32_t mask = __ballot_sync(0xffffffffu, sel);
-      uint32_t base = 0;
-      if (lane == 0 && mask) base = atomicAdd(&sh.out_count, (uint32_t)__popc(mask));
-      base = __shfl_sync(0xffffffffu, base, 0);
-      if (sel) {
-        const uint32_t slot = base + __popc(mask & ((1u << lane) - 1u));
+      if (i < m && key[u] >= key_lo && key[u] <= key_hi && selected(r, key[u], pos[u])) {
         if (slot < (uint32_t)kk) {
           idx_row[slot] = (int32_t)pos[u];
           if (score_row) score_row[slot] = key_to_float(key[u]);
         }
+        ++slot;
       }
     }
   }
+  named_bar_sync(bar_id, NT);   // every thread has read out_count
+  if (tid == 0) sh.out_count = run;
   named_bar_sync(bar_id, NT);
 }
 

@@ -203,7 +203,8 @@ def test_prefill_attention_length_dispatch(lib):
     assert path(1, 2048, 0, 2048, 16, 576, 512, 2048) == dsa.PATH_DENSE_MASKED
     assert path(4, 4096, 0, 4096, 16, 576, 512, 2048) == dsa.PATH_DENSE_MASKED
     assert path(1, 8192, 0, 8192, 16, 576, 512, 2048) == dsa.PATH_GATHER
-    assert path(1, 1024, 3584, 8192, 16, 576, 512, 2048) == dsa.PATH_GATHER    # chunk ends past 4096
+    assert path(1, 6144, 0, 6144, 16, 576, 512, 2048) == dsa.PATH_DENSE_MASKED
+    assert path(1, 1024, 5376, 8192, 16, 576, 512, 2048) == dsa.PATH_GATHER    # chunk ends past 6144
     assert path(1, 512, 0, 512, 4, 64, 64, 16) == dsa.PATH_GATHER              # other head / width
     assert path(1, 0, 0, 16, 16, 576, 512, 16) == dsa.PATH_GATHER
     assert lib.dsa_attn_prefill_workspace(1, 2048, 0, 2048, 16, 576, 512, 2048) >= 256 + 2048 * 32 * 8

@@ -172,12 +172,12 @@ def test_attn_prefill_length_dispatch_gives_the_same_result():
     the gathering path for a long one; on the same selection both equal the
     gathering kernel's output within the attention tolerance."""
     ws = dsa.Workspace("cuda")
-    for kv, q0, nq, k in ((1000, 0, 1000, 128), (4300, 4150, 150, 96)):
+    for kv, q0, nq, k in ((1000, 0, 1000, 128), (6300, 6150, 150, 96)):
         qall, lat = _inputs(1, kv, kv, 11 + kv)
         q = qall[:, q0:q0 + nq].contiguous()
         idx = W.make_selection(1, nq, kv, k, q_offset=q0, seed=kv, device="cuda")
         path = dsa.prefill_attention_path(1, nq, q0, kv, 16, 576, 512, k)
-        assert path == (dsa.PATH_DENSE_MASKED if kv <= 4096 else dsa.PATH_GATHER)
+        assert path == (dsa.PATH_DENSE_MASKED if kv <= 6144 else dsa.PATH_GATHER)
         out, lse = dsa.attn_prefill(q, lat, idx, 512, q_offset=q0, scale=1 / 24, return_lse=True, workspace=ws)
         ref, ref_lse = dsa.sparse_attn_prefill(q, lat, idx, 512, scale=1 / 24, return_lse=True, workspace=ws)
         torch.cuda.synchronize()
