@@ -473,30 +473,43 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const int i = j0 + u * 128 + (int)tid;
             if (i < m) get(i, key[u], pos[u]);
           }
+          // the batch's classes first, then one warp scan of the packed
+          // counts and one pair of shared atomics per warp (per-entry atomics
+          // put a shared-atomic round trip on the chain of every entry)
+          uint32_t abits = 0, obits = 0;
 #pragma unroll
           for (int u = 0; u < kBatch; ++u) {
             const int i = j0 + u * 128 + (int)tid;
             const uint32_t bin = score_bin(key[u]);
-            const bool above = i < m && bin > b0, on = i < m && bin == b0;
-            const uint32_t ma = __ballot_sync(0xffffffffu, above), mo = __ballot_sync(0xffffffffu, on);
-            uint32_t base_a = 0, base_o = 0;
-            if (lane == 0) {
-              if (ma) base_a = atomicAdd(&sel.out_count, (uint32_t)__popc(ma));
-              if (mo) base_o = atomicAdd(&sel.bnd_count, (uint32_t)__popc(mo));
-            }
-            base_a = __shfl_sync(0xffffffffu, base_a, 0);
-            base_o = __shfl_sync(0xffffffffu, base_o, 0);
-            const uint32_t below = (1u << lane) - 1u;
-            if (above) {
-              const uint32_t slot = base_a + __popc(ma & below);
-              if (slot < (uint32_t)kk) {
-                idx_row[slot] = (int32_t)pos[u];
-                if (score_row) score_row[slot] = key_to_float(key[u]);
+            abits |= (i < m && bin > b0) ? (1u << u) : 0u;
+            obits |= (i < m && bin == b0) ? (1u << u) : 0u;
+          }
+          const uint32_t packed = (uint32_t)__popc(abits) | ((uint32_t)__popc(obits) << 16);
+          uint32_t incl = packed;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t2 = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= (uint32_t)o) incl += t2;
+          }
+          uint32_t base_a = 0, base_o = 0;
+          if (lane == 31) {
+            if (incl & 0xFFFFu) base_a = atomicAdd(&sel.out_count, incl & 0xFFFFu);
+            if (incl >> 16) base_o = atomicAdd(&sel.bnd_count, incl >> 16);
+          }
+          const uint32_t excl = incl - packed;
+          uint32_t pa = __shfl_sync(0xffffffffu, base_a, 31) + (excl & 0xFFFFu);
+          uint32_t po = __shfl_sync(0xffffffffu, base_o, 31) + (excl >> 16);
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u) {
+            if ((abits >> u) & 1u) {
+              if (pa < (uint32_t)kk) {
+                idx_row[pa] = (int32_t)pos[u];
+                if (score_row) score_row[pa] = key_to_float(key[u]);
               }
-            }
-            if (on) {
-              const uint32_t slot = base_o + __popc(mo & below);
-              if (slot < (uint32_t)a.cand_cap) bnd[slot] = make_uint2(key[u], pos[u]);
+              ++pa;
+            } else if ((obits >> u) & 1u) {
+              if (po < (uint32_t)a.cand_cap) bnd[po] = make_uint2(key[u], pos[u]);
+              ++po;
             }
           }
         }
