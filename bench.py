@@ -93,17 +93,20 @@ KERNEL_SOURCES = {
 
 
 def measured_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, or None when the
-    summary is missing or the kernel source changed since it was taken."""
+    """(DRAM bytes per launch, captured case or None) from a committed ncu
+    summary; (None, None) when the summary is missing or the kernel source
+    changed since it was taken.  The case names the launch that was captured
+    when it is not a launch of the timed workload itself (a full-size launch
+    too large to capture)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
-        return None
+        return None, None
     with open(p) as f:
         d = json.load(f)
     e = d.get(f"{kernel}:{workload}")
     if not e or e.get("source_hash") != kernel_source_hash(KERNEL_SOURCES[kernel]):
-        return None
-    return e.get("bytes_per_launch")
+        return None, None
+    return e.get("bytes_per_launch"), e.get("case")
 
 
 class ClockSampler:
@@ -866,10 +869,13 @@ def measure_workload(w, args, dev, world, rank, local, steps, warmup, cpu_budget
         tkey = {"indexer_topk_decode": "indexer_scan", "sparse_attn_decode": "latent_attn_decode"}.get(name, name)
         # the training step's selection and attention are the prefill workload's launches
         twl = "prefill" if (w.kind == "train" and name in ("indexer_topk_prefill", "sparse_attn")) else w.name
+        t_bytes, t_case = measured_traffic(tkey, twl)
         kernels[name] = {"bound": bound, "achieved": round(ach, 2), "peak": peak, "unit": wk["unit"],
                          "frac": round(ach / peak, 4), "ms_per_launch": round(t_launch, 4),
-                         "traffic": measured_traffic(tkey, twl),
+                         "traffic": t_bytes,
                          "algorithmic_per_launch": per_launch, "per_unit": wk["per_unit"]}
+        if t_case:
+            kernels[name]["traffic_case"] = t_case
         if bound == "tensor":
             kernels[name]["peak_source"] = (
                 f"sustained bf16 ({peaks['bf16_tflops_sustained']} TFLOP/s: timed inside a {ms:.0f} ms step)"
@@ -888,6 +894,8 @@ def measure_workload(w, args, dev, world, rank, local, steps, warmup, cpu_budget
     dom = max(kernels, key=lambda n: kernels[n]["ms_per_launch"] * max(1, len(seg_ms[n]) // max(1, steps)))
     roof = {k: kernels[dom][k] for k in ("bound", "achieved", "peak", "unit", "frac", "traffic")}
     roof["kernel"] = dom
+    if "traffic_case" in kernels[dom]:
+        roof["traffic_case"] = kernels[dom]["traffic_case"]
     roof["peak_source"] = (f"{peak_src} "
                            f"({kernels[dom].get('peak_source', 'copy bandwidth')}; of {peak_src})")
     if "frac_of_burst" in kernels[dom]:
