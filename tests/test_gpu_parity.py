@@ -520,6 +520,41 @@ def test_decode_selection_with_equal_scores():
     assert not bad, bad[:5]
 
 
+def test_decode_selection_long_rows_exact():
+    """Long ragged sequences (65536, 50001, 32771, 40000, 16385 and 9000
+    cached keys, which take the sampled cut-off of the row top-k) beside a
+    3-key one, and a sequence whose highest scores are 3000 equal keys at its
+    end, so the cut-off falls inside a tie.  Integer values, so the selection
+    is exact (ties to the lower position)."""
+    g = torch.Generator().manual_seed(43)
+    lengths = torch.tensor([65536, 50001, 32771, 40000, 16385, 9000, 3])
+    B, HI, dI, k = lengths.numel(), 16, 64, 2048
+    cu = torch.zeros(B + 1, dtype=torch.int64)
+    cu[1:] = torch.cumsum(lengths, 0)
+    total = int(cu[-1])
+    kc = torch.randint(-3, 4, (total, dI), generator=g).float()
+    # sequence 3: positive queries, and its last 3000 keys all equal to 3, so
+    # they score far above the rest (and tie among themselves)
+    q = torch.randint(-3, 4, (B, HI, dI), generator=g).float()
+    q[3] = q[3].abs() + 1
+    s3 = int(cu[3])
+    kc[s3 + 37000:s3 + 40000] = 3.0
+    w = torch.randint(1, 16, (B, HI), generator=g).float() / 16
+    ws = _ws()
+    idx = dsa.indexer_topk_decode(q.bfloat16().cuda(), w.cuda(), kc.bfloat16().cuda(), cu.cuda(), k, total,
+                                  int(lengths.max()), workspace=ws)
+    torch.cuda.synchronize()
+    _no_device_errors(ws)
+    ref = O.decode_indexer_topk(q.double().numpy(), w.double().numpy(), kc.double().numpy(), cu, k)
+    idx = idx.cpu().numpy()
+    bad = []
+    for b in range(B):
+        bad += checks.topk_exact_errors(idx[b], ref[b], int(lengths[b]) - 1, k)
+    assert not bad, bad[:5]
+    # sequence 3's selection is its raised block's first 2048 keys (ties to the lower position)
+    assert sorted(idx[3]) == list(range(37000, 37000 + k))
+
+
 def test_decode_attention_scattered_and_bad_slots():
     """The decode step's attention (128 heads, 576/512 latent rows: the
     tensor-core kernel whose two CTAs split the latent columns) on ragged
