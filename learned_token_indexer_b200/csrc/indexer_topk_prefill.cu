@@ -84,11 +84,16 @@ __device__ __forceinline__ void raise_floor(const uint32_t* hist, uint32_t k, ui
 // Accumulator plan: each TMEM accumulator holds the heads of kTPA tokens of
 // the block (MMA N = kTPA * HI).  Two tokens per accumulator (four
 // accumulators, one per epilogue warpgroup, which releases it alone) where the
-// MMA shape allows it (N >= 16); four tokens otherwise (two accumulators,
-// every warpgroup reading one token of each).
-template <int HI>
+// MMA shape allows it (N >= 16); four tokens otherwise, and in the wide plan
+// (two accumulators, every warpgroup reading one token of each).  The wide
+// plan halves the MMA instructions and the shared-memory reads of each K^I
+// tile (it is read once per accumulator); measured on B200 with H^I = 64 it
+// is faster with long histories (8192 queries against 32768 keys: 4.91 ->
+// 4.80 ms) and slower with short ones (8192 against 8192: 0.896 -> 0.929 ms),
+// so the launch picks it from the history length.
+template <int HI, bool WIDE>
 struct AccPlan {
-  static constexpr int kTPA = (2 * HI >= 16) ? 2 : 4;
+  static constexpr int kTPA = (WIDE || 2 * HI < 16) ? 4 : 2;
   static constexpr int kNA = kQB / kTPA;
   static constexpr int kNP = kTPA * HI;
 };
@@ -126,12 +131,12 @@ __device__ __forceinline__ bool block_of(const PrefillArgs& a, int r, Block& blk
 
 }  // namespace
 
-template <int HI, bool FP8, int KB, int STAGES>
+template <int HI, bool FP8, int KB, int STAGES, bool WIDE>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     indexer_topk_prefill_kernel(const __grid_constant__ CUtensorMap tmap_q,
                                 const __grid_constant__ CUtensorMap tmap_k, const PrefillArgs a) {
   constexpr int N = kTA * HI;                                 // Q rows per TMA group (4 tokens)
-  using Plan = AccPlan<HI>;
+  using Plan = AccPlan<HI, WIDE>;
   constexpr int kNA = Plan::kNA, kNP = Plan::kNP, kTPA = Plan::kTPA;
   constexpr int kQGroupBytes = N * KB * kSwizzleBytes;
   constexpr int kKBytes = kTileKeys * KB * kSwizzleBytes;
@@ -559,16 +564,19 @@ struct PrefillConfig {
   static constexpr int kSmem = kFixed + STAGES * kKBytes + 2 * STAGES * 8;
 };
 
-template <int HI, bool FP8, int KB>
+template <int HI, bool FP8, int KB, bool WIDE = false>
 static cudaError_t launch_prefill_t(const CUtensorMap& tq, const CUtensorMap& tk, const PrefillArgs& a, int grid,
                                     cudaStream_t stream) {
   using C = PrefillConfig<HI, FP8, KB>;
-  auto kern = indexer_topk_prefill_kernel<HI, FP8, KB, C::STAGES>;
+  auto kern = indexer_topk_prefill_kernel<HI, FP8, KB, C::STAGES, WIDE>;
   cudaError_t e = setup_once_per_device([&]() { return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem); });
   if (e != cudaSuccess) return e;
   kern<<<grid, kPrefillThreads, C::kSmem, stream>>>(tq, tk, a);
   return cudaGetLastError();
 }
+
+// History length from which bf16 H^I = 64 launches take the wide plan.
+constexpr int kWideMinKeys = 16384;
 
 cudaError_t launch_indexer_topk_prefill(int HI, bool fp8, int kblocks, const CUtensorMap& tq,
                                         const CUtensorMap& tk, const PrefillArgs& a, int grid, cudaStream_t stream) {
@@ -576,6 +584,7 @@ cudaError_t launch_indexer_topk_prefill(int HI, bool fp8, int kblocks, const CUt
   case H:                                                                       \
     if (fp8) return launch_prefill_t<H, true, 1>(tq, tk, a, grid, stream);      \
     if (kblocks == 1) return launch_prefill_t<H, false, 1>(tq, tk, a, grid, stream); \
+    if (H == 64 && a.kv_len >= kWideMinKeys) return launch_prefill_t<H, false, 2, true>(tq, tk, a, grid, stream); \
     return launch_prefill_t<H, false, 2>(tq, tk, a, grid, stream);
   switch (HI) {
     DSA_PF_CASE(4)
