@@ -575,7 +575,8 @@ static cudaError_t launch_prefill_t(const CUtensorMap& tq, const CUtensorMap& tk
   return cudaGetLastError();
 }
 
-// History length from which bf16 H^I = 64 launches take the wide plan.
+// History length (keys seen by the chunk's last query) from which bf16
+// H^I = 64 launches take the wide plan.
 constexpr int kWideMinKeys = 16384;
 
 cudaError_t launch_indexer_topk_prefill(int HI, bool fp8, int kblocks, const CUtensorMap& tq,
@@ -584,7 +585,8 @@ cudaError_t launch_indexer_topk_prefill(int HI, bool fp8, int kblocks, const CUt
   case H:                                                                       \
     if (fp8) return launch_prefill_t<H, true, 1>(tq, tk, a, grid, stream);      \
     if (kblocks == 1) return launch_prefill_t<H, false, 1>(tq, tk, a, grid, stream); \
-    if (H == 64 && a.kv_len >= kWideMinKeys) return launch_prefill_t<H, false, 2, true>(tq, tk, a, grid, stream); \
+    if (H == 64 && a.q_offset + a.nq >= kWideMinKeys)                          \
+      return launch_prefill_t<H, false, 2, true>(tq, tk, a, grid, stream);      \
     return launch_prefill_t<H, false, 2>(tq, tk, a, grid, stream);
   switch (HI) {
     DSA_PF_CASE(4)
