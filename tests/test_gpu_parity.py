@@ -201,6 +201,18 @@ def _prefill_exact(w, q_offset=0, nq=None, chunk=None, rows=None):
     assert not bad, bad[:5]
 
 
+def test_prefill_wide_plan_integer_exact():
+    """A chunk whose causal history reaches 16384 keys takes the wide
+    accumulator plan of the fused indexer (bf16, H^I = 64: MMA N = 256, two
+    accumulators of four tokens); the chunk before it, 16381 keys, keeps
+    N = 128.  Integer values, so both are bit-exact against the oracle: every
+    row of the wide chunk (67 rows, a ragged 8-token block at its end) and
+    rows of the other around k and at its end."""
+    w = W.scaled(W.PREFILL, B=1, n=16448, seed=5)
+    rows = [(0, i) for i in range(16381, w.n)] + [(0, i) for i in (0, 2047, 2048, 2049, 8191, 16380)]
+    _prefill_exact(w, chunk=16381, rows=rows)
+
+
 def test_prefill_tiny_exact():
     _prefill_exact(W.TINY)
 
