@@ -900,6 +900,14 @@ def measure_workload(w, args, dev, world, rank, local, steps, warmup, cpu_budget
                            f"({kernels[dom].get('peak_source', 'copy bandwidth')}; of {peak_src})")
     if "frac_of_burst" in kernels[dom]:
         roof["frac_of_burst"] = kernels[dom]["frac_of_burst"]
+    if w.kind == "decode" and all(k["bound"] == "hbm" for k in kernels.values()):
+        # the decode step's scan (+ top-k) and gather together: the step's
+        # algorithmic bytes over the summed event-timed launch durations
+        tot_b = sum(k["algorithmic_per_launch"] for k in kernels.values())
+        tot_ms = sum(k["ms_per_launch"] for k in kernels.values())
+        ach = tot_b / (tot_ms * 1e-3) / 1e9
+        roof["scan_plus_gather"] = {"achieved": round(ach, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                    "frac": round(ach / peaks["hbm_gbs"], 4), "kernels": list(kernels)}
     metric, unit = METRIC[w.kind]
     rec = {
         "metric": metric, "value": job_throughput(world, rows, ms), "unit": unit,
