@@ -82,3 +82,28 @@ def test_sample_rows_cover_the_edges():
     for c0 in range(0, W.LONG.n, W.LONG.chunk):
         assert (0, c0) in rs and (0, c0 + W.LONG.chunk - 1) in rs
     assert len(rows) == len(rs) >= 256
+
+
+def test_traffic_records_name_their_summaries_and_cases():
+    """Every DRAM-traffic record the bench may attach to a roofline names a
+    committed ncu summary; a record taken on another launch than the timed
+    one says which (the long prefill's long-history chunk), and a record is
+    dropped for a workload it was not taken on."""
+    import json
+    import os
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with open(os.path.join(root, "profiles", "traffic.json")) as f:
+        records = json.load(f)
+    for key, rec in records.items():
+        kernel, _, workload = key.partition(":")
+        assert kernel in bench.KERNEL_SOURCES and workload, key
+        assert os.path.exists(os.path.join(root, rec["summary"])), rec["summary"]
+        assert rec["bytes_per_launch"] > 0
+    rec = records["indexer_topk_prefill:long_prefill"]
+    assert "captured launch" in rec["case"]
+    bytes_, case = bench.measured_traffic("indexer_topk_prefill", "long_prefill")
+    if rec["source_hash"] == bench.kernel_source_hash(bench.KERNEL_SOURCES["indexer_topk_prefill"]):
+        assert bytes_ == rec["bytes_per_launch"] and case == rec["case"]
+    else:   # the kernel changed since the capture: no traffic figure
+        assert bytes_ is None and case is None
+    assert bench.measured_traffic("indexer_topk_prefill", "no_such_workload") == (None, None)
